@@ -1,0 +1,202 @@
+"""CPU oracle of the MoE SwiGLU FFN layer -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and its
+Python binding) never loads it and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, loops in the pages' order);
+this module only compiles it with gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+OK, ERR_ARG, ERR_BAD_ID = 0, 1, 3
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, OpenMP, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                               "-fno-fast-math", "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library and return it."""
+    P = ctypes.c_void_p
+    i64, i32 = ctypes.c_int64, ctypes.c_int32
+    lib.oracle_plan.argtypes = [P, P, i64, i32, i32, P, P, P, P, P]
+    lib.oracle_plan.restype = ctypes.c_int
+    lib.oracle_tile_table.argtypes = [P, i32, i32, P, P, P, i64]
+    lib.oracle_tile_table.restype = i64
+    lib.oracle_dispatch.argtypes = [P, P, i64, i64, i32, P]
+    lib.oracle_unpermute_rows.argtypes = [P, P, i64, i64, P]
+    lib.oracle_grouped_gemm.argtypes = [P, P, P, i32, i64, i64, P]
+    lib.oracle_swiglu.argtypes = [P, i64, i64, P]
+    lib.oracle_combine.argtypes = [P, P, P, i64, i64, i32, P]
+    lib.oracle_moe_ffn.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P]
+    lib.oracle_moe_ffn.restype = ctypes.c_int
+    lib.oracle_bruteforce_tokens.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P]
+    lib.oracle_bruteforce_tokens.restype = ctypes.c_int
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = configure(ctypes.CDLL(build()))
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    """bf16 bit patterns as uint16 (accepts a CPU torch bf16 tensor or a uint16 array)."""
+    if isinstance(a, np.ndarray):
+        assert a.dtype == np.uint16
+        return np.ascontiguousarray(a)
+    import torch
+    assert a.dtype == torch.bfloat16 and a.device.type == "cpu"
+    return a.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def plan(ids: np.ndarray, w: np.ndarray | None, E: int):
+    """counts [E], offsets [E+1], perm [R], inv [R], w_sorted [R] (or None)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    M, topk = ids.shape
+    R = M * topk
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    perm = np.zeros(max(R, 1), np.int32)
+    inv = np.zeros(max(R, 1), np.int32)
+    ws = None
+    if w is not None:
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        ws = np.zeros(max(R, 1), np.float32)
+    st = _load().oracle_plan(_p(ids), _p(w) if w is not None else None, M, E, topk,
+                             _p(counts), _p(offsets), _p(perm), _p(inv),
+                             _p(ws) if ws is not None else None)
+    if st != OK:
+        raise OracleError(f"oracle_plan status {st}")
+    return counts, offsets, perm[:R], inv[:R], (ws[:R] if ws is not None else None)
+
+
+def tile_table(offsets: np.ndarray, BM: int):
+    """(expert, row0, row1) per tile, expert by expert."""
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    E = len(offsets) - 1
+    cap = int(offsets[-1]) // BM + E + 1
+    te, r0, r1 = (np.zeros(cap, np.int32) for _ in range(3))
+    n = _load().oracle_tile_table(_p(offsets), E, BM, _p(te), _p(r0), _p(r1), cap)
+    if n < 0:
+        raise OracleError("tile table overflow")
+    return te[:n], r0[:n], r1[:n]
+
+
+def dispatch(x, perm: np.ndarray, topk: int) -> np.ndarray:
+    xb = _u16(x)
+    M, H = xb.shape
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    xp = np.zeros((M * topk, H), np.uint16)
+    _load().oracle_dispatch(_p(xb), _p(perm), M, H, topk, _p(xp))
+    return xp
+
+
+def unpermute_rows(xp, inv: np.ndarray) -> np.ndarray:
+    xb = _u16(xp)
+    R, H = xb.shape
+    inv = np.ascontiguousarray(inv, dtype=np.int32)
+    back = np.zeros((R, H), np.uint16)
+    _load().oracle_unpermute_rows(_p(xb), _p(inv), R, H, _p(back))
+    return back
+
+
+def grouped_gemm(A, B, offsets: np.ndarray) -> np.ndarray:
+    """C fp64 [R, N] = per-expert A_e @ B[e]; A bf16 [R, K], B bf16 [E, K, N]."""
+    Ab, Bb = _u16(A), _u16(B)
+    R, K = Ab.shape
+    E, K2, N = Bb.shape
+    assert K2 == K
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    C = np.zeros((R, N), np.float64)
+    _load().oracle_grouped_gemm(_p(Ab), _p(Bb), _p(offsets), E, K, N, _p(C))
+    return C
+
+
+def swiglu(G: np.ndarray) -> np.ndarray:
+    G = np.ascontiguousarray(G, dtype=np.float64)
+    R, F2 = G.shape
+    h = np.zeros((R, F2 // 2), np.float64)
+    _load().oracle_swiglu(_p(G), R, F2 // 2, _p(h))
+    return h
+
+
+def combine(yp: np.ndarray, inv: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """out fp64 [M, H] = sum_k w[t,k] * yp[inv[t*topk+k]] (yp fp64 [R, H])."""
+    yp = np.ascontiguousarray(yp, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    M, topk = w.shape
+    H = yp.shape[1]
+    inv = np.ascontiguousarray(inv, dtype=np.int32)
+    out = np.zeros((M, H), np.float64)
+    _load().oracle_combine(_p(yp), _p(inv), _p(w), M, H, topk, _p(out))
+    return out
+
+
+def moe_ffn(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The whole layer through the plan; out fp64 [M, H]."""
+    xb, W1b, W2b = _u16(x), _u16(W1), _u16(W2)
+    M, H = xb.shape
+    E, _, F2 = W1b.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    topk = ids.shape[1]
+    out = np.zeros((M, H), np.float64)
+    st = _load().oracle_moe_ffn(_p(xb), _p(W1b), _p(W2b), _p(ids), _p(w), M, H, F2 // 2, E,
+                                topk, _p(out))
+    if st != OK:
+        raise OracleError(f"oracle_moe_ffn status {st}")
+    return out
+
+
+def bruteforce_tokens(x, W1, W2, ids: np.ndarray, w: np.ndarray, tokens) -> np.ndarray:
+    """Rows of the layer output for the listed tokens, computed one token at a time."""
+    xb, W1b, W2b = _u16(x), _u16(W1), _u16(W2)
+    M, H = xb.shape
+    E, _, F2 = W1b.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    topk = ids.shape[1]
+    tok = np.ascontiguousarray(tokens, dtype=np.int64)
+    assert tok.size == 0 or (tok.min() >= 0 and tok.max() < M)
+    out = np.zeros((tok.size, H), np.float64)
+    st = _load().oracle_bruteforce_tokens(_p(xb), _p(W1b), _p(W2b), _p(ids), _p(w), H, F2 // 2, E,
+                                          topk, _p(tok), tok.size, _p(out))
+    if st != OK:
+        raise OracleError(f"oracle_bruteforce_tokens status {st}")
+    return out

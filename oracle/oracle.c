@@ -1,0 +1,343 @@
+/*
+ * oracle.c -- plain, slow, CPU reference of the MoE SwiGLU FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark do.  It shares no code, header or table with the CUDA library.
+ *
+ * Arithmetic: every floating value is carried in fp64.  bf16 inputs are widened
+ * exactly; nothing is rounded back to bf16.  Loops run in the order written, and
+ * the file is compiled with -ffp-contract=off so that two loops that perform the
+ * same operations in the same order give bit-identical fp64 results.
+ *
+ * What it computes (the layer, as the pages state it):
+ *   - PTO MegaMoE article, section "MoE dispatch/combine 为什么慢": the chain is
+ *     a local reorder of routed rows by expert, the expert FFN, and a top-k
+ *     weighted accumulation back into token order.
+ *   - same article, section "MegaMoE 融合算子七阶段": FrontReorder, Dispatch,
+ *     GMM1, SwiGLU, GMM2, Combine, Unpermute.
+ *   - Grouped GEMM article ("Grouped GEMM 为什么适合 MoE"), section "Grouped GEMM
+ *     到底解决什么问题": C_i = A_i x B_i for independent problems i = 0..G-1.
+ *   - same article, section "1. Tiling": each expert's rows cut into tiles of one
+ *     uniform height.
+ *   - COMET paper review, section 4.1.1 (shared tensor decomposition): layer 0
+ *     is independent per token (M), layer 1 couples the top-k rows of a token
+ *     through the reduction.
+ *
+ * Readings taken where the pages are silent (each also listed in the design
+ * notes): SwiGLU is silu(gate) * up with silu(v) = v / (1 + exp(-v)); W1 [E,H,2F]
+ * holds gate in columns [0,F) and up in [F,2F); the permutation is stable in the
+ * flat index i = t*topk + k; gate weights are applied as given (no renormalising).
+ *
+ * Pins (tests that check this file against something other than itself):
+ *   plan            python stable sort of (expert, i); invariants; worked tiling
+ *                   example of the grouped GEMM article
+ *   dispatch        unpermute(permute(x)) = x, bit-exact
+ *   grouped GEMM    numpy float64 matmul per expert
+ *   swiglu          closed form with math.exp on scalars
+ *   layer           E=1,topk=1 equals a dense SwiGLU FFN (torch float64);
+ *                   H=F=1 closed form; identical experts => out = FFN(x) * sum w;
+ *                   linearity in w; per-token brute force equals the plan path
+ *                   bit-exactly
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_BAD_ID 3
+
+static double bf16_widen(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+int oracle_abi_version(void) { return 1; }
+
+/*
+ * Routing plan: per-expert counts, offsets (exclusive prefix sum, E+1 entries),
+ * and the stable permutation of the R = M*topk routed rows.
+ *   perm[s] = i  -- slot s of the expert-ordered buffer holds flat row i = t*topk+k
+ *   inv[i]  = s  -- inverse of perm
+ *   w_sorted[s] = w[perm[s]]
+ * Within one expert the slots follow ascending i (a counting sort).
+ */
+int oracle_plan(const int32_t *ids, const float *w, int64_t M, int32_t E, int32_t topk,
+                int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                float *w_sorted)
+{
+    if (M < 0 || E < 1 || topk < 1 || topk > E)
+        return ORACLE_ERR_ARG;
+    int64_t R = M * (int64_t)topk;
+    for (int64_t i = 0; i < R; i++)
+        if (ids[i] < 0 || ids[i] >= E)
+            return ORACLE_ERR_BAD_ID;
+
+    for (int32_t e = 0; e < E; e++)
+        counts[e] = 0;
+    for (int64_t i = 0; i < R; i++)
+        counts[ids[i]] += 1;
+
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; e++)
+        offsets[e + 1] = offsets[e] + counts[e];
+
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (!cursor)
+        return ORACLE_ERR_ARG;
+    for (int32_t e = 0; e < E; e++)
+        cursor[e] = offsets[e];
+    for (int64_t i = 0; i < R; i++) {
+        int32_t s = cursor[ids[i]]++;
+        perm[s] = (int32_t)i;
+        inv[i] = s;
+    }
+    free(cursor);
+    if (w_sorted && w)
+        for (int64_t s = 0; s < R; s++)
+            w_sorted[s] = w[perm[s]];
+    return ORACLE_OK;
+}
+
+/*
+ * Tiling of the grouped problem: every expert's row segment [offsets[e],
+ * offsets[e+1]) is cut into tiles of BM rows; the last tile of an expert may be
+ * short, an expert with no rows has no tile.  Tiles are listed expert by expert,
+ * top to bottom.  Returns the number of tiles, or -1 if max_tiles is too small.
+ */
+int64_t oracle_tile_table(const int32_t *offsets, int32_t E, int32_t BM,
+                          int32_t *tile_expert, int32_t *tile_row0, int32_t *tile_row1,
+                          int64_t max_tiles)
+{
+    int64_t n = 0;
+    for (int32_t e = 0; e < E; e++) {
+        for (int32_t r = offsets[e]; r < offsets[e + 1]; r += BM) {
+            if (n >= max_tiles)
+                return -1;
+            tile_expert[n] = e;
+            tile_row0[n] = r;
+            tile_row1[n] = (r + BM < offsets[e + 1]) ? r + BM : offsets[e + 1];
+            n++;
+        }
+    }
+    return n;
+}
+
+/* Dispatch (permute): xp[s, :] = x[perm[s] / topk, :]; a copy of bf16 bits. */
+void oracle_dispatch(const uint16_t *x, const int32_t *perm, int64_t M, int64_t H,
+                     int32_t topk, uint16_t *xp)
+{
+    int64_t R = M * (int64_t)topk;
+    for (int64_t s = 0; s < R; s++) {
+        int64_t t = perm[s] / topk;
+        memcpy(xp + s * H, x + t * H, sizeof(uint16_t) * (size_t)H);
+    }
+}
+
+/* Unpermute of a copy: x_back[i, :] = xp[inv[i], :] for flat rows i. */
+void oracle_unpermute_rows(const uint16_t *xp, const int32_t *inv, int64_t R, int64_t H,
+                           uint16_t *x_back)
+{
+    for (int64_t i = 0; i < R; i++)
+        memcpy(x_back + i * H, xp + (int64_t)inv[i] * H, sizeof(uint16_t) * (size_t)H);
+}
+
+/*
+ * Grouped GEMM: for every expert e and every row s of its segment,
+ *   C[s, n] = sum_{k=0}^{K-1} A[s, k] * B[e, k, n]      (k ascending)
+ * A bf16 [R, K] row-major, B bf16 [E, K, N] row-major, C fp64 [R, N].
+ */
+void oracle_grouped_gemm(const uint16_t *A, const uint16_t *B, const int32_t *offsets,
+                         int32_t E, int64_t K, int64_t N, double *C)
+{
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *Be = B + (int64_t)e * K * N;
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t s = offsets[e]; s < offsets[e + 1]; s++) {
+            double *c = C + s * N;
+            for (int64_t n = 0; n < N; n++)
+                c[n] = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double a = bf16_widen(A[s * K + k]);
+                const uint16_t *b = Be + k * N;
+                for (int64_t n = 0; n < N; n++)
+                    c[n] += a * bf16_widen(b[n]);
+            }
+        }
+    }
+}
+
+/* SwiGLU on a gate|up row block: h[s, j] = silu(G[s, j]) * G[s, F + j]. */
+void oracle_swiglu(const double *G, int64_t R, int64_t F, double *h)
+{
+    for (int64_t s = 0; s < R; s++)
+        for (int64_t j = 0; j < F; j++)
+            h[s * F + j] = silu(G[s * 2 * F + j]) * G[s * 2 * F + F + j];
+}
+
+/*
+ * Combine of expert-ordered, unweighted rows:
+ *   out[t, c] = sum_{k=0}^{topk-1} w[t, k] * yp[inv[t*topk + k], c]   (k ascending)
+ */
+void oracle_combine(const double *yp, const int32_t *inv, const float *w, int64_t M,
+                    int64_t H, int32_t topk, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; t++) {
+        double *o = out + t * H;
+        for (int64_t c = 0; c < H; c++)
+            o[c] = 0.0;
+        for (int32_t k = 0; k < topk; k++) {
+            int64_t i = t * topk + k;
+            double wk = (double)w[i];
+            const double *y = yp + (int64_t)inv[i] * H;
+            for (int64_t c = 0; c < H; c++)
+                o[c] += wk * y[c];
+        }
+    }
+}
+
+/*
+ * One expert's FFN on one bf16 row v [H]:
+ *   g = v . W1[e]            (2F values, sum over h ascending)
+ *   a[j] = silu(g[j]) * g[F + j]
+ *   y = a . W2[e]            (H values, sum over j ascending)
+ * scratch must hold 2F + F doubles.
+ */
+static void expert_ffn_row(const uint16_t *v, const uint16_t *W1e, const uint16_t *W2e,
+                           int64_t H, int64_t F, double *scratch, double *y)
+{
+    double *g = scratch;
+    double *a = scratch + 2 * F;
+    for (int64_t j = 0; j < 2 * F; j++)
+        g[j] = 0.0;
+    for (int64_t h = 0; h < H; h++) {
+        double xv = bf16_widen(v[h]);
+        const uint16_t *wrow = W1e + h * 2 * F;
+        for (int64_t j = 0; j < 2 * F; j++)
+            g[j] += xv * bf16_widen(wrow[j]);
+    }
+    for (int64_t j = 0; j < F; j++)
+        a[j] = silu(g[j]) * g[F + j];
+    for (int64_t c = 0; c < H; c++)
+        y[c] = 0.0;
+    for (int64_t j = 0; j < F; j++) {
+        const uint16_t *wrow = W2e + j * H;
+        for (int64_t c = 0; c < H; c++)
+            y[c] += a[j] * bf16_widen(wrow[c]);
+    }
+}
+
+/*
+ * The whole layer through the plan, stage by stage:
+ *   plan -> dispatch -> per expert (GEMM1, SwiGLU, GEMM2) on its row segment ->
+ *   weighted combine back to token order (k ascending).
+ * out fp64 [M, H].  Returns an ORACLE_* status.
+ */
+int oracle_moe_ffn(const uint16_t *x, const uint16_t *W1, const uint16_t *W2,
+                   const int32_t *ids, const float *w, int64_t M, int64_t H, int64_t F,
+                   int32_t E, int32_t topk, double *out)
+{
+    int64_t R = M * (int64_t)topk;
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *perm = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    uint16_t *xp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(R ? R * H : 1));
+    double *yp = (double *)malloc(sizeof(double) * (size_t)(R ? R * H : 1));
+    int st = ORACLE_ERR_ARG;
+    if (!counts || !offsets || !perm || !inv || !xp || !yp)
+        goto done;
+    st = oracle_plan(ids, w, M, E, topk, counts, offsets, perm, inv, NULL);
+    if (st != ORACLE_OK)
+        goto done;
+    oracle_dispatch(x, perm, M, H, topk, xp);
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *W1e = W1 + (int64_t)e * H * 2 * F;
+        const uint16_t *W2e = W2 + (int64_t)e * F * H;
+#pragma omp parallel
+        {
+            double *scratch = (double *)malloc(sizeof(double) * (size_t)(3 * F));
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t s = offsets[e]; s < offsets[e + 1]; s++)
+                expert_ffn_row(xp + s * H, W1e, W2e, H, F, scratch, yp + s * H);
+            free(scratch);
+        }
+    }
+    oracle_combine(yp, inv, w, M, H, topk, out);
+done:
+    free(counts);
+    free(offsets);
+    free(perm);
+    free(inv);
+    free(xp);
+    free(yp);
+    return st;
+}
+
+/*
+ * Brute force, no plan: for each listed token t,
+ *   out_rows[j, :] = sum_{k ascending} w[t, k] * FFN_{ids[t, k]}(x[t])
+ * with the same per-row arithmetic as oracle_moe_ffn, so the two agree bit for
+ * bit.  Used on small cases as a cross-check and on large cases to compute a
+ * sample of output rows one by one.
+ */
+int oracle_bruteforce_tokens(const uint16_t *x, const uint16_t *W1, const uint16_t *W2,
+                             const int32_t *ids, const float *w, int64_t H, int64_t F,
+                             int32_t E, int32_t topk, const int64_t *tokens, int64_t n_tokens,
+                             double *out_rows)
+{
+    for (int64_t j = 0; j < n_tokens; j++)
+        for (int32_t k = 0; k < topk; k++) {
+            int32_t e = ids[tokens[j] * topk + k];
+            if (e < 0 || e >= E)
+                return ORACLE_ERR_BAD_ID;
+        }
+#pragma omp parallel
+    {
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)(3 * F));
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t j = 0; j < n_tokens; j++) {
+            int64_t t = tokens[j];
+            double *o = out_rows + j * H;
+            for (int64_t c = 0; c < H; c++)
+                o[c] = 0.0;
+            for (int32_t k = 0; k < topk; k++) {
+                int32_t e = ids[t * topk + k];
+                expert_ffn_row(x + t * H, W1 + (int64_t)e * H * 2 * F,
+                               W2 + (int64_t)e * F * H, H, F, scratch, y);
+                double wk = (double)w[t * topk + k];
+                for (int64_t c = 0; c < H; c++)
+                    o[c] += wk * y[c];
+            }
+        }
+        free(scratch);
+        free(y);
+    }
+    return ORACLE_OK;
+}
+
+/* Number of OpenMP threads the oracle's parallel loops use. */
+int oracle_num_threads(void)
+{
+    int n = 1;
+#ifdef _OPENMP
+#pragma omp parallel
+    {
+#pragma omp single
+        n = omp_get_num_threads();
+    }
+#endif
+    return n;
+}

@@ -1,0 +1,81 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check that the
+pins of test_oracle_pins.py catch every one of them.
+
+Each mutant is a one-line edit of oracle.c compiled into a temporary library; the
+pin functions then run against it in a child process (a mutant that writes out of
+bounds may crash, which also counts as caught).  A mutant that passes every pin
+would show a hole in the pins.
+"""
+import os
+import subprocess
+import sys
+import textwrap
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+TESTS = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(TESTS)
+
+MUTANTS = {
+    "gate_up_swapped": ("a[j] = silu(g[j]) * g[F + j];", "a[j] = silu(g[F + j]) * g[j];"),
+    "silu_sign": ("v / (1.0 + exp(-v))", "v / (1.0 + exp(v))"),
+    "weight_dropped_in_combine": ("o[c] += wk * y[c];\n        }\n    }\n}",
+                                  "o[c] += y[c];\n        }\n    }\n}"),
+    "unstable_scatter": ("for (int64_t i = 0; i < R; i++) {\n        int32_t s = cursor",
+                         "for (int64_t i = R - 1; i >= 0; i--) {\n        int32_t s = cursor"),
+    "offsets_off_by_one": ("offsets[e + 1] = offsets[e] + counts[e];",
+                           "offsets[e + 1] = offsets[e] + counts[e] + (e == 0);"),
+    "dispatch_wrong_token": ("int64_t t = perm[s] / topk;", "int64_t t = perm[s] % topk;"),
+    "gemm_transposed_b": ("c[n] += a * bf16_widen(b[n]);",
+                          "c[n] += a * bf16_widen(Be[(n % K) * N + (k % N)]);"),
+    "w2_row_index": ("const uint16_t *wrow = W2e + j * H;",
+                     "const uint16_t *wrow = W2e + (F - 1 - j) * H;"),
+    "tile_short_edge": ("tile_row1[n] = (r + BM < offsets[e + 1]) ? r + BM : offsets[e + 1];",
+                        "tile_row1[n] = r + BM;"),
+}
+
+CHILD = textwrap.dedent("""
+    import ctypes, sys
+    sys.path[:0] = [{root!r}, {tests!r}]
+    import oracle
+    oracle._lib = oracle.configure(ctypes.CDLL({lib!r}))
+    import test_oracle_pins as pins
+    calls = [
+        lambda: pins.test_plan_matches_stable_sort(33, 8, 2, True),
+        lambda: pins.test_plan_matches_stable_sort(50, 5, 3, False),
+        pins.test_tiling_worked_example,
+        pins.test_tile_table_brute_force,
+        pins.test_dispatch_and_unpermute_identity,
+        pins.test_grouped_gemm_matches_numpy_matmul,
+        pins.test_swiglu_closed_form,
+        pins.test_dense_special_case_e1_topk1,
+        pins.test_scalar_closed_form_h1_f1,
+        pins.test_identical_experts_sum_of_weights,
+        pins.test_layer_matches_torch_per_token_mixture,
+    ]
+    caught = 0
+    for c in calls:
+        try:
+            c()
+        except Exception:
+            caught += 1
+    sys.exit(0 if caught == 0 else 3)
+""")
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site of {name} not unique"
+    mpath = tmp_path / "mutant.c"
+    mpath.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                           "-std=c11", "-w", "-o", str(lib), str(mpath), "-lm"])
+    child = CHILD.format(root=ROOT, tests=TESTS, lib=str(lib))
+    r = subprocess.run([sys.executable, "-c", child], capture_output=True, timeout=300)
+    assert r.returncode != 0, f"mutant {name} passed every pin"
