@@ -1,0 +1,395 @@
+#!/usr/bin/env python3
+"""Benchmark of the MoE SwiGLU FFN layer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--n-c -1]
+    python bench.py --impl reference ...      # the CPU oracle on the host cores
+
+A step is one pass of the whole layer (plan -> dispatch -> GEMM1+SwiGLU -> GEMM2
++gate-weighted scatter -> combine) over one batch of M tokens, through the
+public call moe_ffn_fused.  Inputs are seeded and synthetic (grouped_gemm_plan_b200
+.workload); weights are resident in HBM.  L2 is flushed (a 256 MiB write)
+before every timed step, outside the timed events.  With N GPUs every rank runs
+its own batch (its own seed): tokens are independent, so the layer shards with
+no collective on the data path (weak scaling); the only collectives are the
+barrier and the max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "MoE-layer tokens/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral")
+    ap.add_argument("--n-c", type=int, default=-1, dest="n_c")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+def peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- oracle arm
+
+def oracle_tokens_per_s(wl, seconds: float):
+    """Time the CPU oracle (per-token brute force, all host cores) on a bounded sample."""
+    import oracle
+    from grouped_gemm_plan_b200 import workload as W
+    x = W.make_x(wl)
+    W1, W2 = W.make_weights(wl)
+    ids, tw = W.make_routing(wl)
+    t0 = time.perf_counter()
+    oracle.bruteforce_tokens(x, W1, W2, ids, tw, np.arange(1))
+    one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(wl.M, seconds / one)))
+    tokens = np.arange(n) * max(1, wl.M // n)
+    tokens = tokens[tokens < wl.M]
+    t0 = time.perf_counter()
+    oracle.bruteforce_tokens(x, W1, W2, ids, tw, tokens)
+    dt = time.perf_counter() - t0
+    return len(tokens) / dt, len(tokens), dt, oracle.num_threads()
+
+
+def run_reference(args):
+    from grouped_gemm_plan_b200 import workload as W
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.WORKLOADS[args.workload]
+    import oracle
+    oracle.build()
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    vals = []
+    n_tok = 0
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        v, n, dt, cores = oracle_tokens_per_s(wl, per_step if i >= args.warmup else 0.5)
+        if i >= args.warmup:
+            vals.append(v)
+            n_tok = n
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wl.M / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "H": wl.H, "F": wl.F, "E": wl.E,
+                   "topk": wl.topk, "routing": wl.routing, "seed": wl.seed},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} tokens per step of the {wl.name} batch, per-token "
+                                   f"brute force in fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rows = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "grouped_gemm_plan_b200", "csrc", "grouped_gemm.cu")
+    sha = source_sha(src)
+    for r in rows:
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from grouped_gemm_plan_b200 import binding as B
+    from grouped_gemm_plan_b200 import workload as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    B.load()
+
+    wl = W.rank_workload(W.WORKLOADS[args.workload], rank)
+    M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
+    x_h = W.make_x(wl).pin_memory()
+    ids_np, tw_np = W.make_routing(wl)
+    ids_h = torch.from_numpy(ids_np).pin_memory()
+    tw_h = torch.from_numpy(tw_np).pin_memory()
+    W1 = torch.empty((E, H, 2 * F), dtype=torch.bfloat16, device=dev)
+    W2 = torch.empty((E, F, H), dtype=torch.bfloat16, device=dev)
+    W.make_weights(wl, W1, W2)
+    x = x_h.to(dev)
+    ids = ids_h.to(dev)
+    tw = tw_h.to(dev)
+    out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(R, dtype=torch.int32, device=dev)
+    ws = B.alloc_workspace(B.OP_FFN_FUSED, M, H, F, E, topk, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=args.n_c)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    st = B.moe_get_device_status(ws)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} after warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each, device time by CUDA events
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(1)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    st = B.moe_get_device_status(ws)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} in the timed region")
+
+    # ---- stage breakdown (same kernels as the n_c = 0 path, one call per stage)
+    inv = torch.empty(R, dtype=torch.int32, device=dev)
+    w_sorted = torch.empty(R, dtype=torch.float32, device=dev)
+    xp = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
+    hbuf = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
+    yk = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
+    small_ws = B.alloc_workspace(B.OP_PLAN, M, H, F, E, topk, dev)
+    names = ["plan", "dispatch", "gemm1_swiglu", "gemm2_scatter", "combine"]
+    calls = [
+        lambda: B.moe_plan(ids, tw, E, counts, offsets, perm, inv, w_sorted, small_ws),
+        lambda: B.moe_dispatch(x, perm, topk, xp, small_ws),
+        lambda: B.moe_grouped_gemm(xp, W1, offsets, B.EPI_SWIGLU, hbuf, small_ws),
+        lambda: B.moe_grouped_gemm(hbuf, W2, offsets, B.EPI_WEIGHT_SCATTER, yk, small_ws,
+                                   w_sorted=w_sorted, perm=perm),
+        lambda: B.moe_combine(yk, None, None, M, topk, out, small_ws),
+    ]
+    stage_ms = {n: [] for n in names}
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        evs[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            evs[j + 1].record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            for j, n in enumerate(names):
+                stage_ms[n].append(evs[j].elapsed_time(evs[j + 1]))
+    assert B.moe_get_device_status(small_ws) == B.MOE_OK
+    stage_avg = {n: statistics.mean(v) for n, v in stage_ms.items()}
+
+    # ---- end to end: pinned host inputs in, result out, every step
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    out_h = torch.empty((M, H), dtype=torch.bfloat16).pin_memory()
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(1)
+        e2e_ev[i][0].record(stream)
+        x.copy_(x_h, non_blocking=True)
+        ids.copy_(ids_h, non_blocking=True)
+        tw.copy_(tw_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * M * args.steps / (total_ms / 1e3)
+    e2e_value = world * M * args.steps / (e2e_ms / 1e3)
+
+    pk, pk_kind = peaks()
+    flops_g1 = 4.0 * R * H * F
+    g1_s = stage_avg["gemm1_swiglu"] / 1e3
+    achieved = flops_g1 / g1_s / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    traffic = measured_traffic("gemm1_swiglu", wl.name)
+    roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue", "bound": "tensor",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{pk_kind} bf16_tflops_sustained", "traffic": traffic,
+                "algorithmic": f"4*R*H*F = {flops_g1:.4g} FLOP per launch"}
+    g2 = 2.0 * R * H * F / (stage_avg["gemm2_scatter"] / 1e3) / 1e12
+    disp_bytes = M * H * 2 + R * H * 2 + R * 4
+    comb_bytes = R * H * 2 + M * H * 2
+    extra = {
+        "stages_ms": stage_avg,
+        "gemm1_tflops": achieved, "gemm2_tflops": g2,
+        "grouped_gemm_frac_of_bf16_peak": {"gemm1": achieved / peak, "gemm2": g2 / peak},
+        "dispatch_gbs": disp_bytes / (stage_avg["dispatch"] / 1e3) / 1e9,
+        "combine_gbs": comb_bytes / (stage_avg["combine"] / 1e3) / 1e9,
+        "hbm_peak_gbs": pk["hbm_gbs"],
+        "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        v, n, dt, cores = oracle_tokens_per_s(W.WORKLOADS[args.workload], args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} tokens of the {wl.name} batch, per-token brute force in fp64, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "M": M, "H": H, "F": F, "E": E, "topk": topk,
+                       "routing": wl.routing, "std": wl.std, "seed": W.WORKLOADS[args.workload].seed,
+                       "n_c": args.n_c, "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (independent batches, no collective)"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 5 * args.steps,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+            **extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+"""Thin Python binding of libmoe.so: argument marshalling only.
+
+Every function here has the name and the meaning of the C entry point it wraps
+(include/moe.h); it takes torch tensors that already live on the GPU, passes
+their device pointers and the current CUDA stream, and raises MoEError on a
+non-zero status.  No step of the layer runs in Python or on the CPU: if the
+library is missing, importing this module's functions fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+MOE_OK = 0
+(MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_BAD_EXPERT_ID, MOE_ERR_WORKSPACE_TOO_SMALL,
+ MOE_ERR_TIMEOUT, MOE_ERR_CUDA, MOE_ERR_MISALIGNED, MOE_ERR_BAD_INDEX) = range(1, 9)
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+                3: "MOE_ERR_BAD_EXPERT_ID", 4: "MOE_ERR_WORKSPACE_TOO_SMALL",
+                5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_MISALIGNED",
+                8: "MOE_ERR_BAD_INDEX"}
+
+EPI_STORE, EPI_SWIGLU, EPI_WEIGHT_SCATTER = 0, 1, 2
+OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED = 0, 1, 2, 3, 4
+
+# Every symbol include/moe.h declares.
+EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_plan", "moe_dispatch",
+           "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_get_device_status",
+           "moe_set_wait_timeout_ns", "moe_last_error"]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(path: str | None = None):
+    """Load libmoe.so (built in-tree by grouped_gemm_plan_b200.build). Raises if absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _build.LIB
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with `python -m grouped_gemm_plan_b200.build` "
+                          "(there is no fallback implementation)")
+    lib = ctypes.CDLL(p)
+    P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    st = ctypes.c_int
+    lib.moe_abi_version.restype = ctypes.c_int
+    lib.moe_workspace_size.argtypes = [ctypes.c_int, i64, i64, i64, i32, i32]
+    lib.moe_workspace_size.restype = sz
+    lib.moe_plan.argtypes = [P, P, i64, i32, i32, P, P, P, P, P, P, sz, P]
+    lib.moe_plan.restype = st
+    lib.moe_dispatch.argtypes = [P, P, i64, i64, i32, P, P, sz, P]
+    lib.moe_dispatch.restype = st
+    lib.moe_grouped_gemm.argtypes = [P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P, P, P, sz, P]
+    lib.moe_grouped_gemm.restype = st
+    lib.moe_combine.argtypes = [P, P, P, i64, i64, i32, P, P, sz, P]
+    lib.moe_combine.restype = st
+    lib.moe_ffn_fused.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]
+    lib.moe_ffn_fused.restype = st
+    lib.moe_get_device_status.argtypes = [P, P]
+    lib.moe_get_device_status.restype = st
+    lib.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.moe_set_wait_timeout_ns.restype = None
+    lib.moe_last_error.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libmoe must be on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int):
+    if status != MOE_OK:
+        raise MoEError(status, load().moe_last_error().decode())
+
+
+def moe_abi_version() -> int:
+    return int(load().moe_abi_version())
+
+
+def moe_workspace_size(op: int, M: int, H: int, F: int, E: int, topk: int) -> int:
+    return int(load().moe_workspace_size(op, M, H, F, E, topk))
+
+
+def alloc_workspace(op: int, M: int, H: int, F: int, E: int, topk: int, device) -> torch.Tensor:
+    """A zeroed uint8 workspace of the size the op needs (torch allocations are 256-byte aligned)."""
+    n = moe_workspace_size(op, M, H, F, E, topk)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_plan(topk_ids, topk_w, E, counts, offsets, perm, inv_perm, w_sorted, ws, stream=None):
+    M, topk = topk_ids.shape
+    _check(load().moe_plan(_ptr(topk_ids), _ptr(topk_w), M, E, topk, _ptr(counts), _ptr(offsets),
+                           _ptr(perm), _ptr(inv_perm), _ptr(w_sorted), _ptr(ws), ws.numel(),
+                           _stream(stream)))
+
+
+def moe_dispatch(x, perm, topk, xp, ws, stream=None):
+    M, H = x.shape
+    _check(load().moe_dispatch(_ptr(x), _ptr(perm), M, H, topk, _ptr(xp), _ptr(ws), ws.numel(),
+                               _stream(stream)))
+
+
+def moe_grouped_gemm(A, B, offsets, epi, C, ws, w_sorted=None, perm=None, stream=None):
+    R, K = A.shape
+    E, K2, N = B.shape
+    if K2 != K:
+        raise ValueError(f"A has K={K} but B has K={K2}")
+    _check(load().moe_grouped_gemm(_ptr(A), _ptr(B), _ptr(offsets), E, R, K, N, epi,
+                                   _ptr(w_sorted), _ptr(perm), _ptr(C), _ptr(ws), ws.numel(),
+                                   _stream(stream)))
+
+
+def moe_combine(y, inv_perm, topk_w, M, topk, out, ws, stream=None):
+    H = y.shape[1]
+    _check(load().moe_combine(_ptr(y), _ptr(inv_perm), _ptr(topk_w), M, H, topk, _ptr(out),
+                              _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_ffn_fused(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, ws, n_c=0,
+                  stream=None):
+    M, H = x.shape
+    E, _, F2 = W1.shape
+    topk = topk_ids.shape[1]
+    _check(load().moe_ffn_fused(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w), M, H,
+                                F2 // 2, E, topk, n_c, _ptr(out), _ptr(counts), _ptr(offsets),
+                                _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    """Synchronises the stream; returns the device status word and clears it."""
+    return int(load().moe_get_device_status(_ptr(ws), _stream(stream)))
+
+
+def moe_set_wait_timeout_ns(ns: int) -> None:
+    load().moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_last_error() -> str:
+    return load().moe_last_error().decode()

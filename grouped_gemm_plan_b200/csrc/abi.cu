@@ -1,0 +1,289 @@
+// abi.cu -- the extern "C" entry points of libmoe.so (declared in include/moe.h).
+//
+// Host-side work only: argument validation (before anything is launched),
+// workspace carving, and kernel launches on the caller's stream.  Every step of
+// the layer itself runs in the kernels of plan.cu, permute.cu and
+// grouped_gemm.cu; there is no host or CPU fallback.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
+                        int32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
+                            void* xp, int32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_combine(const void* y, const int32_t* inv, const float* w, int64_t M,
+                           int64_t H, int32_t topk, void* out, int32_t* status, int num_sms,
+                           cudaStream_t stream);
+int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, int32_t E,
+                        int64_t R, int64_t K, int64_t N, int epi, const float* w_sorted,
+                        const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
+                        int num_sms, cudaStream_t stream);
+}  // namespace moe
+
+namespace {
+
+thread_local std::string g_last_error;
+uint64_t g_timeout_ns = 2000000000ull;
+
+constexpr size_t kCtrlBytes = 256;
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
+
+moe_status fail(moe_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+moe_status fail(moe_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+moe_status cuda_fail(cudaError_t err, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+int32_t* status_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
+
+// Intermediates of moe_ffn_fused inside the workspace.
+struct FusedLayout {
+  size_t xp, h, yk, w_sorted, total;
+};
+
+FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t topk) {
+  const int64_t R = M * topk;
+  FusedLayout L;
+  size_t off = kCtrlBytes;
+  L.xp = off;
+  off += align256(size_t(R) * size_t(H) * 2);
+  L.h = off;
+  off += align256(size_t(R) * size_t(F) * 2);
+  L.yk = off;
+  off += align256(size_t(R) * size_t(H) * 2);
+  L.w_sorted = off;
+  off += align256(size_t(R) * 4);
+  L.total = off;
+  return L;
+}
+
+moe_status check_ws(moe_op op, void* ws, size_t ws_bytes, int64_t M, int64_t H, int64_t F,
+                    int32_t E, int32_t topk) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MOE_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  const size_t need = moe_workspace_size(op, M, H, F, E, topk);
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return MOE_OK;
+}
+
+moe_status check_route(int64_t M, int32_t E, int32_t topk) {
+  if (M < 0) return fail(MOE_ERR_INVALID_ARG, "M = %lld < 0", (long long)M);
+  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E = %d < 1", E);
+  if (E > MOE_MAX_EXPERTS)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d > %d", E, MOE_MAX_EXPERTS);
+  if (topk < 1 || topk > E) return fail(MOE_ERR_INVALID_ARG, "topk = %d not in [1, E=%d]", topk, E);
+  if (topk > 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "topk = %d > 32", topk);
+  if (M * topk > kMaxRows) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "M*topk exceeds 2^31-1");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns > 0 ? ns : 1; }
+
+size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
+  (void)E;
+  if (M < 0 || H < 0 || F < 0 || topk < 0) return kCtrlBytes;
+  if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, topk).total;
+  return kCtrlBytes;
+}
+
+moe_status moe_get_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t err = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, sizeof v, s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_get_device_status");
+  return static_cast<moe_status>(v);
+}
+
+moe_status moe_plan(const int32_t* topk_ids, const float* topk_w, int64_t M, int32_t E,
+                    int32_t topk, int32_t* counts, int32_t* offsets, int32_t* perm,
+                    int32_t* inv_perm, float* w_sorted, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  if (counts == nullptr || offsets == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  if (M > 0 && (topk_ids == nullptr || perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "topk_ids and perm must not be NULL");
+  if (w_sorted != nullptr && topk_w == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "w_sorted requested without topk_w");
+  st = check_ws(MOE_OP_PLAN, ws, ws_bytes, M, 0, 0, E, topk);
+  if (st != MOE_OK) return st;
+  cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(M * topk), E, counts,
+                                     offsets, perm, inv_perm, w_sorted, status_word(ws),
+                                     num_sms_current(), reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_plan launch");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
+                        void* xp, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (M < 0 || topk < 1 || topk > 32 || M * topk > kMaxRows)
+    return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
+  if (H <= 0 || H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 8", (long long)H);
+  moe_status st = check_ws(MOE_OP_DISPATCH, ws, ws_bytes, M, H, 0, 1, topk);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  if (x == nullptr || perm == nullptr || xp == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "x, perm and xp must not be NULL");
+  if (!aligned16(x) || !aligned16(xp)) return fail(MOE_ERR_MISALIGNED, "x and xp must be 16-byte aligned");
+  cudaError_t err = moe::launch_dispatch(x, perm, M, H, topk, xp, status_word(ws), num_sms_current(),
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_dispatch launch");
+  return MOE_OK;
+}
+
+moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk_w, int64_t M,
+                       int64_t H, int32_t topk, void* out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  g_last_error.clear();
+  if (M < 0 || topk < 1 || topk > 32 || M * topk > kMaxRows)
+    return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
+  if (H <= 0 || H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 8", (long long)H);
+  moe_status st = check_ws(MOE_OP_COMBINE, ws, ws_bytes, M, H, 0, 1, topk);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  if (y == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "y and out must not be NULL");
+  if (!aligned16(y) || !aligned16(out)) return fail(MOE_ERR_MISALIGNED, "y and out must be 16-byte aligned");
+  cudaError_t err = moe::launch_combine(y, inv_perm, topk_w, M, H, topk, out, status_word(ws),
+                                        num_sms_current(), reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_combine launch");
+  return MOE_OK;
+}
+
+moe_status moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets, int32_t E,
+                            int64_t R, int64_t K, int64_t N, moe_epilogue epi,
+                            const float* w_sorted, const int32_t* perm, void* C, void* ws,
+                            size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64", (long long)K);
+  if (N <= 0 || N % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "N = %lld must be a positive multiple of 64", (long long)N);
+  if (epi != MOE_EPI_STORE && epi != MOE_EPI_SWIGLU && epi != MOE_EPI_WEIGHT_SCATTER)
+    return fail(MOE_ERR_INVALID_ARG, "unknown epilogue %d", (int)epi);
+  if (epi == MOE_EPI_SWIGLU && (N / 2) % 64 != 0)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "SWIGLU needs N/2 = %lld a multiple of 64", (long long)(N / 2));
+  if (K > (int64_t(1) << 30) || N > (int64_t(1) << 30) || E * K > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N too large");
+  moe_status st = check_ws(MOE_OP_GROUPED_GEMM, ws, ws_bytes, R, N, K, E, 1);
+  if (st != MOE_OK) return st;
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets must not be NULL");
+  if (R == 0) return MOE_OK;
+  if (A == nullptr || B == nullptr || C == nullptr) return fail(MOE_ERR_INVALID_ARG, "A, B and C must not be NULL");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return fail(MOE_ERR_MISALIGNED, "A, B and C must be 16-byte aligned");
+  if (epi == MOE_EPI_WEIGHT_SCATTER && (w_sorted == nullptr || perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "WEIGHT_SCATTER needs w_sorted and perm");
+  const int rc = moe::launch_grouped_gemm(A, B, offsets, E, R, K, N, static_cast<int>(epi), w_sorted,
+                                          perm, C, status_word(ws), g_timeout_ns, num_sms_current(),
+                                          reinterpret_cast<cudaStream_t>(stream));
+  if (rc == 1) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_grouped_gemm launch");
+  return MOE_OK;
+}
+
+moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
+                         const float* topk_w, int64_t M, int64_t H, int64_t F, int32_t E,
+                         int32_t topk, int32_t n_c, void* out, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                         void* stream) {
+  g_last_error.clear();
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  if (H <= 0 || H % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 64", (long long)H);
+  if (F <= 0 || F % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be a positive multiple of 64", (long long)F);
+  if (H > (int64_t(1) << 30) || F > (int64_t(1) << 29) || int64_t(E) * H > kMaxRows || int64_t(E) * F > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
+  if (n_c < -1) return fail(MOE_ERR_INVALID_ARG, "n_c = %d < -1", n_c);
+  st = check_ws(MOE_OP_FFN_FUSED, ws, ws_bytes, M, H, F, E, topk);
+  if (st != MOE_OK) return st;
+  if (counts == nullptr || offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  if (M == 0) {
+    // Still a defined plan: zero counts and offsets.
+    cudaStream_t s0 = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = moe::launch_plan(topk_ids, topk_w, 0, E, counts, offsets, perm, nullptr,
+                                       nullptr, status_word(ws), num_sms_current(), s0);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ffn_fused plan");
+  }
+  if (x == nullptr || W1 == nullptr || W2 == nullptr || topk_ids == nullptr || topk_w == nullptr ||
+      out == nullptr || perm == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "x, W1, W2, topk_ids, topk_w, out and perm must not be NULL");
+  if (!aligned16(x) || !aligned16(W1) || !aligned16(W2) || !aligned16(out))
+    return fail(MOE_ERR_MISALIGNED, "x, W1, W2 and out must be 16-byte aligned");
+
+  const int64_t R = M * topk;
+  const FusedLayout L = fused_layout(M, H, F, topk);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* xp = base + L.xp;
+  void* h = base + L.h;
+  void* yk = base + L.yk;
+  float* w_sorted = reinterpret_cast<float*>(base + L.w_sorted);
+  int32_t* status = status_word(ws);
+  const int sms = num_sms_current();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
+                                     perm, nullptr, w_sorted, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused plan");
+  err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused dispatch");
+  int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,
+                                    nullptr, h, status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM1)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM1");
+  rc = moe::launch_grouped_gemm(h, W2, offsets, E, R, F, H, MOE_EPI_WEIGHT_SCATTER, w_sorted, perm,
+                                yk, status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM2)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM2");
+  err = moe::launch_combine(yk, nullptr, nullptr, M, H, topk, out, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused combine");
+  return MOE_OK;
+}
+
+}  // extern "C"

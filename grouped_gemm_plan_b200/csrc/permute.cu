@@ -1,0 +1,150 @@
+// permute.cu -- dispatch (gather into expert order) and combine (top-k reduction
+// back to token order).  Both are HBM-bound copies of bf16 rows; neither has a
+// contraction, so they stay off the tensor cores.
+//
+// Dispatch is the permute of the PTO MegaMoE article ("MegaMoE 融合算子七阶段":
+// Dispatch) and COMET's layer-0 token dispatch (COMET review, section 3.2).
+// Combine is the top-k weighted accumulation ("MoE dispatch/combine 为什么慢":
+// topK 加权累加) plus Unpermute.
+//
+// Layout of the work: one warp per output row; each lane moves 16-byte vectors
+// (8 bf16), 32 lanes cover 512 contiguous bytes per step, so every access is a
+// full, coalesced 128-byte line.  Grids are a multiple of the SM count with 8
+// warps per CTA; rows are walked grid-stride.  Combine reads the top-k source
+// vectors of a step before it accumulates, so up to topk loads per lane are in
+// flight; the sum runs in fp32 registers in ascending k, one bf16 cast at the end.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int PM_THREADS = 256;
+
+__global__ void __launch_bounds__(PM_THREADS)
+    dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int32_t R,
+                    int32_t topk, int32_t vpr, uint4* __restrict__ xp, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int32_t nwarps = (gridDim.x * PM_THREADS) >> 5;
+  for (int32_t s = (blockIdx.x * PM_THREADS + threadIdx.x) >> 5; s < R; s += nwarps) {
+    const int32_t i = __ldg(perm + s);
+    uint4* dst = xp + static_cast<int64_t>(s) * vpr;
+    if (i < 0 || i >= R) {
+      if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+      for (int32_t c = lane; c < vpr; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const uint4* src = x + static_cast<int64_t>(i / topk) * vpr;
+    int32_t c = lane;
+    for (; c + 96 < vpr; c += 128) {
+      const uint4 a0 = __ldg(src + c), a1 = __ldg(src + c + 32), a2 = __ldg(src + c + 64),
+                  a3 = __ldg(src + c + 96);
+      dst[c] = a0;
+      dst[c + 32] = a1;
+      dst[c + 64] = a2;
+      dst[c + 96] = a3;
+    }
+    for (; c < vpr; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float wk) {
+  const float2 p0 = unpack_bf16x2(v.x), p1 = unpack_bf16x2(v.y), p2 = unpack_bf16x2(v.z),
+               p3 = unpack_bf16x2(v.w);
+  acc[0] = fmaf(wk, p0.x, acc[0]);
+  acc[1] = fmaf(wk, p0.y, acc[1]);
+  acc[2] = fmaf(wk, p1.x, acc[2]);
+  acc[3] = fmaf(wk, p1.y, acc[3]);
+  acc[4] = fmaf(wk, p2.x, acc[4]);
+  acc[5] = fmaf(wk, p2.y, acc[5]);
+  acc[6] = fmaf(wk, p3.x, acc[6]);
+  acc[7] = fmaf(wk, p3.y, acc[7]);
+}
+
+// out[t] = bf16(sum_k w[t,k] * y[row(t,k)]), row(t,k) = inv ? inv[t*topk+k] : t*topk+k.
+template <int KMAX>
+__global__ void __launch_bounds__(PM_THREADS)
+    combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
+                   const float* __restrict__ w, int32_t M, int32_t R, int32_t topk,
+                   int32_t vpr, uint4* __restrict__ out, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int32_t nwarps = (gridDim.x * PM_THREADS) >> 5;
+  for (int32_t t = (blockIdx.x * PM_THREADS + threadIdx.x) >> 5; t < M; t += nwarps) {
+    int32_t my_row = 0;
+    float my_w = 1.0f;
+    if (lane < topk) {
+      const int32_t i = t * topk + lane;
+      my_row = inv != nullptr ? __ldg(inv + i) : i;
+      if (w != nullptr) my_w = __ldg(w + i);
+      if (my_row < 0 || my_row >= R) {
+        set_status(status, MOE_ERR_BAD_INDEX);
+        my_row = -1;
+      }
+    }
+    int32_t rows[KMAX];
+    float wk[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+      wk[k] = __shfl_sync(0xffffffffu, my_w, k);
+    }
+    uint4* dst = out + static_cast<int64_t>(t) * vpr;
+    for (int32_t c = lane; c < vpr; c += 32) {
+      uint4 v[KMAX];
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k)
+        v[k] = (k < topk && rows[k] >= 0) ? __ldg(y + static_cast<int64_t>(rows[k]) * vpr + c)
+                                          : make_uint4(0, 0, 0, 0);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k)
+        if (k < topk) acc_bf16x8(acc, v[k], wk[k]);
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      dst[c] = o;
+    }
+  }
+}
+
+static int grid_for_rows(int64_t rows, int num_sms) {
+  const int64_t per_cta = PM_THREADS / 32;
+  const int64_t want = (rows + per_cta - 1) / per_cta;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
+                            void* xp, int32_t* status, int num_sms, cudaStream_t stream) {
+  const int64_t R = M * topk;
+  if (R == 0) return cudaSuccess;
+  dispatch_kernel<<<grid_for_rows(R, num_sms), PM_THREADS, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
+      static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y, const int32_t* inv, const float* w, int64_t M,
+                           int64_t H, int32_t topk, void* out, int32_t* status, int num_sms,
+                           cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  const int grid = grid_for_rows(M, num_sms);
+  const int32_t R = static_cast<int32_t>(M * topk);
+  const int32_t vpr = static_cast<int32_t>(H / 8);
+  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  uint4* ov = reinterpret_cast<uint4*>(out);
+  const int32_t m = static_cast<int32_t>(M);
+  if (topk <= 2)
+    combine_kernel<2><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 4)
+    combine_kernel<4><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 8)
+    combine_kernel<8><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 16)
+    combine_kernel<16><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  else
+    combine_kernel<32><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

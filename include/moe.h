@@ -1,0 +1,196 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE SwiGLU FFN layer library (libmoe.so).
+ *
+ * The layer: given routed tokens (top-k expert ids and gate weights per token),
+ * reorder the routed rows by expert, run every expert's SwiGLU FFN on its rows
+ * as one grouped GEMM pair, and sum each token's top-k results back in token
+ * order, weighted by its gate weights.
+ *
+ * Sources (pages the method is taken from):
+ *   [PTO]   "PTO MoE算子实战dispatch/combine如何与计算流水线重叠实现性能倍增",
+ *           sections "MoE dispatch/combine 为什么慢" (reorder by expert -> expert
+ *           FFN -> top-k weighted accumulation) and "MegaMoE 融合算子七阶段"
+ *           (FrontReorder, Dispatch, GMM1, SwiGLU, GMM2, Combine, Unpermute).
+ *   [GG]    "Grouped GEMM 为什么适合 MoE？从碎片小矩阵到通信友好的算子设计",
+ *           sections "Grouped GEMM 到底解决什么问题" (C_i = A_i x B_i with
+ *           per-problem sizes; a fixed set of CTAs pulls tiles from one queue),
+ *           "1. Tiling", "2. Double-buffer pipeline", "Fused GemmAdd" (fp32
+ *           epilogue arithmetic, one cast on output).
+ *   [COMET] "COMET: Fine-grained Computation-communication Overlapping for
+ *           Mixture-of-Experts" (paper review), sections 4.1 (shared-tensor
+ *           decomposition and rescheduling) and 4.2 (thread-block specialisation,
+ *           adaptive thread-block count n_c chosen from profiled metadata).
+ *
+ * Conventions for every call
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *     caller allocates and owns all buffers.  The library allocates no device
+ *     memory and keeps no device state between calls.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream) and does not synchronise.
+ *   - Errors that the host can see (null pointers, bad sizes, misalignment,
+ *     unsupported shapes, short workspace) return before anything is launched;
+ *     moe_last_error() then gives a one-line message (thread-local).
+ *   - Errors that only the device can see (an expert id out of [0, E), a wait
+ *     that ran out of time) are recorded in the status word at the start of the
+ *     workspace; read it with moe_get_device_status().  Kernels never trap.
+ *   - bf16 tensors are row-major with the stated shapes and dense rows; every
+ *     base pointer must be 16-byte aligned.  Integers are int32, weights fp32.
+ *   - R = M * topk is the number of routed rows.  Flat routed index i = t*topk+k.
+ *   - M = 0 is legal: nothing is launched and MOE_OK is returned.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, negative size, topk > E, ...      */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* H or F not a multiple of 64, E > MOE_MAX_EXPERTS */
+  MOE_ERR_BAD_EXPERT_ID = 3,      /* device: some topk_ids entry is outside [0, E)   */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  MOE_ERR_TIMEOUT = 5,            /* device: a bounded wait ran out                   */
+  MOE_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed                */
+  MOE_ERR_MISALIGNED = 7,         /* a base pointer is not 16-byte aligned            */
+  MOE_ERR_BAD_INDEX = 8           /* device: a permutation entry is outside [0, R)    */
+} moe_status;
+
+/* Largest expert count the kernels accept. */
+#define MOE_MAX_EXPERTS 1024
+
+/* Epilogue of moe_grouped_gemm ([GG] "Fused GemmAdd": the accumulator is kept in
+ * fp32 and transformed before the single cast to bf16 on output). */
+typedef enum moe_epilogue {
+  /* C[s, n] = bf16(acc[s, n]);  C is [R, N]. */
+  MOE_EPI_STORE = 0,
+  /* B = W1 holds gate columns [0, N/2) and up columns [N/2, N);
+   * C[s, j] = bf16(silu(acc[s, j]) * acc[s, N/2 + j]),  silu(v) = v / (1 + e^-v);
+   * C is [R, N/2].  ([PTO] "MegaMoE 融合算子七阶段": SwiGLU consumes GMM1's
+   * output as soon as it is produced.) */
+  MOE_EPI_SWIGLU = 1,
+  /* C[perm[s], n] = bf16(w_sorted[s] * acc[s, n]): the gate-weighted row goes
+   * straight to its token-major slot i = t*topk + k; C is [R, N]. */
+  MOE_EPI_WEIGHT_SCATTER = 2
+} moe_epilogue;
+
+/* Which call a workspace is sized for. */
+typedef enum moe_op {
+  MOE_OP_PLAN = 0,
+  MOE_OP_DISPATCH = 1,
+  MOE_OP_GROUPED_GEMM = 2,
+  MOE_OP_COMBINE = 3,
+  MOE_OP_FFN_FUSED = 4
+} moe_op;
+
+/* Version of this ABI (incremented on any incompatible change). */
+int moe_abi_version(void);
+
+/* Bytes of device workspace `op` needs for this shape (always >= 256; the first
+ * 256 bytes hold the device status word).  The workspace must be 256-byte
+ * aligned.  Its contents need no initialisation except that the status word
+ * should read 0 before the first call (zero the buffer once, or call
+ * moe_get_device_status once, which clears it). */
+size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
+
+/*
+ * moe_plan -- routing plan ([PTO] "MegaMoE 融合算子七阶段", FrontReorder; [GG]
+ * "Grouped GEMM 到底解决什么问题": per-problem sizes passed as arrays).
+ *   topk_ids  int32 [M, topk]   expert of each routed row
+ *   topk_w    fp32  [M, topk]   gate weight of each routed row (may be NULL if
+ *                               w_sorted is NULL)
+ *   counts    int32 [E]         out: rows routed to each expert
+ *   offsets   int32 [E+1]       out: exclusive prefix sum, offsets[E] = R
+ *   perm      int32 [R]         out: perm[s] = i, the flat routed row held in
+ *                               expert-ordered slot s; stable: within one expert
+ *                               the slots follow ascending i
+ *   inv_perm  int32 [R]         out: inv_perm[perm[s]] = s (may be NULL)
+ *   w_sorted  fp32  [R]         out: w_sorted[s] = topk_w[perm[s]] (may be NULL)
+ * Duplicate ids within a token are legal and counted twice.  If any id is out of
+ * [0, E), the device status becomes MOE_ERR_BAD_EXPERT_ID, counts and offsets
+ * are all zero and perm/inv_perm are the identity (safe for later calls).
+ */
+moe_status moe_plan(const int32_t* topk_ids, const float* topk_w, int64_t M, int32_t E,
+                    int32_t topk, int32_t* counts, int32_t* offsets, int32_t* perm,
+                    int32_t* inv_perm, float* w_sorted, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * moe_dispatch -- permute ([PTO] Dispatch; [COMET] 3.2, layer 0 token dispatch):
+ *   xp[s, :] = x[perm[s] / topk, :]          x bf16 [M, H], xp bf16 [R, H]
+ * A pure copy of bf16 bits.  H must be a multiple of 8.  A perm entry outside
+ * [0, R) writes a zero row and records MOE_ERR_BAD_INDEX.
+ */
+moe_status moe_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
+                        void* xp, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_grouped_gemm -- one persistent tcgen05 kernel for every expert's GEMM
+ * ([GG] "Grouped GEMM 到底解决什么问题"):
+ *   for every expert e and row s in [offsets[e], offsets[e+1]):
+ *     acc[s, n] = sum_k A[s, k] * B[e, k, n]     (fp32 accumulate)
+ *   then the epilogue `epi` writes C (see moe_epilogue).
+ *   A bf16 [R, K] (rows in expert order), B bf16 [E, K, N] row-major (N
+ *   contiguous), offsets int32 [E+1] as written by moe_plan.
+ *   w_sorted, perm: used by MOE_EPI_WEIGHT_SCATTER only (else may be NULL).
+ * K and N must be multiples of 64 (for SWIGLU, N/2 must be a multiple of 64).
+ */
+moe_status moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets, int32_t E,
+                            int64_t R, int64_t K, int64_t N, moe_epilogue epi,
+                            const float* w_sorted, const int32_t* perm, void* C, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine -- top-k reduction back to token order ([PTO] "MoE dispatch/combine
+ * 为什么慢": topK 加权累加; Combine + Unpermute):
+ *   out[t, :] = bf16( sum_{k=0}^{topk-1} wk * fp32(y[row(t, k), :]) )   (k ascending)
+ *   row(t, k) = inv_perm[t*topk + k] if inv_perm != NULL (y in expert order),
+ *               t*topk + k           if inv_perm == NULL (y token-major, as
+ *                                    written by MOE_EPI_WEIGHT_SCATTER)
+ *   wk = topk_w[t*topk + k] if topk_w != NULL, else 1.
+ *   y bf16 [R, H], out bf16 [M, H]; H a multiple of 8.
+ */
+moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk_w, int64_t M,
+                       int64_t H, int32_t topk, void* out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * moe_ffn_fused -- the whole layer:
+ *   out[t, :] = sum_k topk_w[t, k] * FFN_{topk_ids[t, k]}(x[t, :])
+ *   FFN_e(v) = (silu(v . W1[e][:, :F]) * (v . W1[e][:, F:])) . W2[e]
+ *   x bf16 [M, H], W1 bf16 [E, H, 2F], W2 bf16 [E, F, H], out bf16 [M, H].
+ * It runs plan -> dispatch -> GEMM1 with the SwiGLU epilogue -> GEMM2 with the
+ * gate-weight scatter epilogue -> combine.  counts [E], offsets [E+1] and perm
+ * [R] receive the plan (as moe_plan).  The intermediates (expert-ordered x, the
+ * SwiGLU activations, the weighted expert outputs) live in the workspace
+ * (moe_workspace_size(MOE_OP_FFN_FUSED, ...)).
+ *   n_c: thread blocks given to the memory stages (dispatch / combine) while the
+ *   GEMM blocks run, [COMET] 4.2.2.  0 runs the stages as consecutive kernels;
+ *   -1 takes the value from the library's profiled table for this shape.
+ * H and F must be multiples of 64.
+ */
+moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
+                         const float* topk_w, int64_t M, int64_t H, int64_t F, int32_t E,
+                         int32_t topk, int32_t n_c, void* out, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Synchronises `stream`, returns the device status word of `ws` (a moe_status)
+ * and clears it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error. */
+moe_status moe_get_device_status(void* ws, void* stream);
+
+/* Time limit, in nanoseconds, of every bounded device-side wait (default 2 s). */
+void moe_set_wait_timeout_ns(uint64_t ns);
+
+/* Message of the last host-side error on this thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

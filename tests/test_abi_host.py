@@ -1,0 +1,132 @@
+"""The C ABI on the host: the library loads, exports every symbol include/moe.h
+declares, and rejects bad arguments before launching anything (no GPU needed:
+validation runs before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_gemm_plan_b200 import binding as B
+from grouped_gemm_plan_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert header_functions() == sorted(B.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(B.library_path())
+    for name in header_functions():
+        assert hasattr(raw, name), f"{name} missing from libmoe.so"
+
+
+def test_abi_version(lib):
+    assert B.moe_abi_version() == 1
+
+
+def test_workspace_sizes(lib):
+    for op in (B.OP_PLAN, B.OP_DISPATCH, B.OP_GROUPED_GEMM, B.OP_COMBINE):
+        assert B.moe_workspace_size(op, 4096, 4096, 14336, 8, 2) == 256
+    R, H, F = 8192, 4096, 14336
+    fused = B.moe_workspace_size(B.OP_FFN_FUSED, 4096, H, F, 8, 2)
+    assert fused >= 256 + 2 * R * H * 2 + R * F * 2 + R * 4
+    assert B.moe_workspace_size(B.OP_FFN_FUSED, 0, H, F, 8, 2) == 256
+
+
+FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
+FAKE_WS = ctypes.c_void_p(0x20000)     # 256-byte aligned
+
+
+def _err(lib):
+    return lib.moe_last_error().decode()
+
+
+def test_plan_validation(lib):
+    # topk > E
+    st = lib.moe_plan(FAKE, FAKE, 4, 2, 3, FAKE, FAKE, FAKE, None, None, FAKE_WS, 256, None)
+    assert st == 1 and "topk" in _err(lib)
+    # E too large
+    st = lib.moe_plan(FAKE, FAKE, 4, 2000, 2, FAKE, FAKE, FAKE, None, None, FAKE_WS, 256, None)
+    assert st == 2
+    # negative M
+    assert lib.moe_plan(FAKE, FAKE, -1, 8, 2, FAKE, FAKE, FAKE, None, None, FAKE_WS, 256, None) == 1
+    # null counts
+    assert lib.moe_plan(FAKE, FAKE, 4, 8, 2, None, FAKE, FAKE, None, None, FAKE_WS, 256, None) == 1
+    # workspace too small / misaligned / null
+    assert lib.moe_plan(FAKE, FAKE, 4, 8, 2, FAKE, FAKE, FAKE, None, None, FAKE_WS, 100, None) == 4
+    assert lib.moe_plan(FAKE, FAKE, 4, 8, 2, FAKE, FAKE, FAKE, None, None,
+                        ctypes.c_void_p(0x20010), 256, None) == 7
+    assert lib.moe_plan(FAKE, FAKE, 4, 8, 2, FAKE, FAKE, FAKE, None, None, None, 256, None) == 1
+    # w_sorted without topk_w
+    assert lib.moe_plan(FAKE, None, 4, 8, 2, FAKE, FAKE, FAKE, None, FAKE, FAKE_WS, 256, None) == 1
+
+
+def test_gemm_validation(lib):
+    g = lib.moe_grouped_gemm
+    ok = dict(E=8, R=256, K=256, N=512)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return g(kw.get("A", FAKE), FAKE, FAKE, a["E"], a["R"], a["K"], a["N"], kw.get("epi", 0),
+                 kw.get("w", None), kw.get("perm", None), FAKE, FAKE_WS, 256, None)
+    assert call(K=100) == 2
+    assert call(N=96) == 2
+    assert call(epi=1, N=192) == 2            # N/2 = 96 not a multiple of 64
+    assert call(epi=7) == 1
+    assert call(E=0) == 2
+    assert call(R=-1) == 1
+    assert call(epi=2) == 1                    # scatter without w_sorted/perm
+    assert call(A=ctypes.c_void_p(0x10008)) == 7
+
+
+def test_dispatch_combine_validation(lib):
+    assert lib.moe_dispatch(FAKE, FAKE, 4, 100, 2, FAKE, FAKE_WS, 256, None) == 2   # H % 8
+    assert lib.moe_dispatch(FAKE, FAKE, 4, 64, 0, FAKE, FAKE_WS, 256, None) == 1    # topk
+    assert lib.moe_dispatch(ctypes.c_void_p(0x10004), FAKE, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 7
+    assert lib.moe_dispatch(None, FAKE, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 1
+    assert lib.moe_combine(FAKE, FAKE, FAKE, 4, 64, 2, None, FAKE_WS, 256, None) == 1
+    assert lib.moe_combine(FAKE, FAKE, FAKE, 4, 64, 33, FAKE, FAKE_WS, 256, None) == 1
+    # M = 0 is a no-op even with null data pointers
+    assert lib.moe_dispatch(None, None, 0, 64, 2, None, FAKE_WS, 256, None) == 0
+    assert lib.moe_combine(None, None, None, 0, 64, 2, None, FAKE_WS, 256, None) == 0
+
+
+def test_fused_validation(lib):
+    f = lib.moe_ffn_fused
+    need = B.moe_workspace_size(B.OP_FFN_FUSED, 16, 128, 128, 4, 2)
+    args = lambda **kw: [FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("M", 16), kw.get("H", 128),
+                         kw.get("F", 128), kw.get("E", 4), kw.get("topk", 2), kw.get("n_c", 0),
+                         FAKE, FAKE, FAKE, FAKE, FAKE_WS, kw.get("ws", need), None]
+    assert f(*args(H=100)) == 2
+    assert f(*args(F=96)) == 2
+    assert f(*args(topk=5)) == 1
+    assert f(*args(n_c=-2)) == 1
+    assert f(*args(ws=need - 1)) == 4
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.moe_dispatch(x, torch.zeros(8, dtype=torch.int32), 2, x, torch.zeros(256, dtype=torch.uint8))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        B.load(str(tmp_path / "nope.so"))
