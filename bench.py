@@ -20,6 +20,8 @@ import datetime
 import hashlib
 import json
 import os
+import shutil
+import signal
 import statistics
 import subprocess
 import sys
@@ -76,10 +78,12 @@ class ClockSampler:
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            cmd = ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                   "--format=csv,noheader,nounits", "-lms", "200"]
+            if shutil.which("stdbuf"):
+                cmd = ["stdbuf", "-oL"] + cmd      # one line per sample, not one block at exit
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True, bufsize=1)
         except OSError:
             self.proc = None
             return
@@ -93,11 +97,13 @@ class ClockSampler:
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
+        time.sleep(0.3)                      # one more sample period
+        self.proc.send_signal(signal.SIGINT)
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+            self.proc.wait(timeout=5)
         if self.thread:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
@@ -121,23 +127,29 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- oracle arm
 
-def oracle_tokens_per_s(wl, seconds: float):
-    """Time the CPU oracle (per-token brute force, all host cores) on a bounded sample."""
-    import oracle
+def oracle_inputs(wl):
     from grouped_gemm_plan_b200 import workload as W
     x = W.make_x(wl)
     W1, W2 = W.make_weights(wl)
     ids, tw = W.make_routing(wl)
+    return x, W1, W2, ids, tw
+
+
+def oracle_tokens_per_s(wl, seconds: float, inputs=None):
+    """Time the CPU oracle (per-token brute force, all host cores) on a bounded sample."""
+    import oracle
+    x, W1, W2, ids, tw = inputs if inputs is not None else oracle_inputs(wl)
+    cores = oracle.num_threads()
     t0 = time.perf_counter()
-    oracle.bruteforce_tokens(x, W1, W2, ids, tw, np.arange(1))
-    one = max(time.perf_counter() - t0, 1e-4)
-    n = int(max(1, min(wl.M, seconds / one)))
+    oracle.bruteforce_tokens(x, W1, W2, ids, tw, np.arange(min(cores, wl.M)))
+    per_token = max(time.perf_counter() - t0, 1e-4) / min(cores, wl.M)   # all cores busy
+    n = int(max(1, min(wl.M, seconds / per_token)))
     tokens = np.arange(n) * max(1, wl.M // n)
     tokens = tokens[tokens < wl.M]
     t0 = time.perf_counter()
     oracle.bruteforce_tokens(x, W1, W2, ids, tw, tokens)
     dt = time.perf_counter() - t0
-    return len(tokens) / dt, len(tokens), dt, oracle.num_threads()
+    return len(tokens) / dt, len(tokens), dt, cores
 
 
 def run_reference(args):
@@ -149,11 +161,12 @@ def run_reference(args):
     import oracle
     oracle.build()
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    inputs = oracle_inputs(wl)
     vals = []
     n_tok = 0
     cores = 1
     for i in range(args.warmup + args.steps):
-        v, n, dt, cores = oracle_tokens_per_s(wl, per_step if i >= args.warmup else 0.5)
+        v, n, dt, cores = oracle_tokens_per_s(wl, per_step if i >= args.warmup else 0.5, inputs)
         if i >= args.warmup:
             vals.append(v)
             n_tok = n
@@ -273,7 +286,7 @@ def run_ours(args):
     w_sorted = torch.empty(R, dtype=torch.float32, device=dev)
     xp = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
     hbuf = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
-    yk = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
+    yk = torch.empty((R, H), dtype=torch.float32, device=dev)
     small_ws = B.alloc_workspace(B.OP_PLAN, M, H, F, E, topk, dev)
     names = ["plan", "dispatch", "gemm1_swiglu", "gemm2_scatter", "combine"]
     calls = [
@@ -339,7 +352,7 @@ def run_ours(args):
                 "algorithmic": f"4*R*H*F = {flops_g1:.4g} FLOP per launch"}
     g2 = 2.0 * R * H * F / (stage_avg["gemm2_scatter"] / 1e3) / 1e12
     disp_bytes = M * H * 2 + R * H * 2 + R * 4
-    comb_bytes = R * H * 2 + M * H * 2
+    comb_bytes = R * H * 4 + M * H * 2
     extra = {
         "stages_ms": stage_avg,
         "gemm1_tflops": achieved, "gemm2_tflops": g2,

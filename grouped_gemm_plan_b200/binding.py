@@ -66,7 +66,7 @@ def load(path: str | None = None):
     lib.moe_dispatch.restype = st
     lib.moe_grouped_gemm.argtypes = [P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P, P, P, sz, P]
     lib.moe_grouped_gemm.restype = st
-    lib.moe_combine.argtypes = [P, P, P, i64, i64, i32, P, P, sz, P]
+    lib.moe_combine.argtypes = [P, i32, P, P, i64, i64, i32, P, P, sz, P]
     lib.moe_combine.restype = st
     lib.moe_ffn_fused.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]
     lib.moe_ffn_fused.restype = st
@@ -138,9 +138,13 @@ def moe_grouped_gemm(A, B, offsets, epi, C, ws, w_sorted=None, perm=None, stream
 
 
 def moe_combine(y, inv_perm, topk_w, M, topk, out, ws, stream=None):
+    """y is bf16 or fp32 [R, H] (the dtype of the tensor selects the C flag)."""
     H = y.shape[1]
-    _check(load().moe_combine(_ptr(y), _ptr(inv_perm), _ptr(topk_w), M, H, topk, _ptr(out),
-                              _ptr(ws), ws.numel(), _stream(stream)))
+    if y.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("moe_combine takes bf16 or fp32 rows")
+    _check(load().moe_combine(_ptr(y), 1 if y.dtype == torch.float32 else 0, _ptr(inv_perm),
+                              _ptr(topk_w), M, H, topk, _ptr(out), _ptr(ws), ws.numel(),
+                              _stream(stream)))
 
 
 def moe_ffn_fused(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, ws, n_c=0,

@@ -17,9 +17,9 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
                         int32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream);
-cudaError_t launch_combine(const void* y, const int32_t* inv, const float* w, int64_t M,
-                           int64_t H, int32_t topk, void* out, int32_t* status, int num_sms,
-                           cudaStream_t stream);
+cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
+                           int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
+                           int num_sms, cudaStream_t stream);
 int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, int32_t E,
                         int64_t R, int64_t K, int64_t N, int epi, const float* w_sorted,
                         const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
@@ -82,8 +82,8 @@ FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t topk) {
   off += align256(size_t(R) * size_t(H) * 2);
   L.h = off;
   off += align256(size_t(R) * size_t(F) * 2);
-  L.yk = off;
-  off += align256(size_t(R) * size_t(H) * 2);
+  L.yk = off;  // fp32: the weighted rows are summed once more before the bf16 cast
+  off += align256(size_t(R) * size_t(H) * 4);
   L.w_sorted = off;
   off += align256(size_t(R) * 4);
   L.total = off;
@@ -179,9 +179,9 @@ moe_status moe_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H
   return MOE_OK;
 }
 
-moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk_w, int64_t M,
-                       int64_t H, int32_t topk, void* out, void* ws, size_t ws_bytes,
-                       void* stream) {
+moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
+                       const float* topk_w, int64_t M, int64_t H, int32_t topk, void* out,
+                       void* ws, size_t ws_bytes, void* stream) {
   g_last_error.clear();
   if (M < 0 || topk < 1 || topk > 32 || M * topk > kMaxRows)
     return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
@@ -191,8 +191,10 @@ moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk
   if (M == 0) return MOE_OK;
   if (y == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "y and out must not be NULL");
   if (!aligned16(y) || !aligned16(out)) return fail(MOE_ERR_MISALIGNED, "y and out must be 16-byte aligned");
-  cudaError_t err = moe::launch_combine(y, inv_perm, topk_w, M, H, topk, out, status_word(ws),
-                                        num_sms_current(), reinterpret_cast<cudaStream_t>(stream));
+  if (y_fp32 != 0 && y_fp32 != 1) return fail(MOE_ERR_INVALID_ARG, "y_fp32 must be 0 or 1");
+  cudaError_t err = moe::launch_combine(y, y_fp32 != 0, inv_perm, topk_w, M, H, topk, out,
+                                        status_word(ws), num_sms_current(),
+                                        reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "moe_combine launch");
   return MOE_OK;
 }
@@ -281,7 +283,7 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
                                 yk, status, g_timeout_ns, sms, s);
   if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM2)")
                               : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM2");
-  err = moe::launch_combine(yk, nullptr, nullptr, M, H, topk, out, status, sms, s);
+  err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused combine");
   return MOE_OK;
 }

@@ -17,7 +17,8 @@
 //   warp 0       one thread issues TMA loads (A tile 128x64, B tile 64x256)
 //   warp 1       allocates TMEM (512 columns); one thread issues tcgen05.mma
 //   warps 2..5   epilogue: tcgen05.ld (one TMEM lane = one output row per thread),
-//                fp32 math, bf16 stores
+//                fp32 math, bf16 stores (fp32 stores for the gate-weighted scatter,
+//                whose rows are summed once more by the combine)
 //
 // Tile order: expert by expert; inside an expert, n-tile outer, m-tile inner, so
 // the CTAs running at the same time share one B column block (read from HBM
@@ -59,7 +60,8 @@ struct GemmArgs {
   int32_t up_col;     // SWIGLU: first up column of B (= F)
   const float* w_sorted;
   const int32_t* perm;
-  __nv_bfloat16* C;
+  __nv_bfloat16* C;   // bf16 output (STORE, SWIGLU)
+  float* Cf;          // fp32 output (WEIGHT_SCATTER)
   int64_t ldc;
   int32_t* status;
   uint64_t timeout_ns;
@@ -106,6 +108,14 @@ __device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const float 
     u.w = pack_bf16x2(v[8 * q + 6] * scale, v[8 * q + 7] * scale);
     d[q] = u;
   }
+}
+
+__device__ __forceinline__ void store_row_chunk_f32(float* dst, const float (&v)[32], float scale) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    d[q] = make_float4(v[4 * q] * scale, v[4 * q + 1] * scale, v[4 * q + 2] * scale,
+                       v[4 * q + 3] * scale);
 }
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
@@ -327,14 +337,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           }
           drow = dest;
         }
-        __nv_bfloat16* dst = args.C + drow * args.ldc;
 #pragma unroll 1
         for (int c = 0; c < G_BN / 32; ++c) {
           float v[32];
           tmem_ld32(t_row + c * 32, v);
           tmem_ld_wait();
           const int32_t col = tc.ni * G_BN + c * 32;
-          if (ok && col < args.n_out) store_row_chunk(dst + col, v, scale);
+          if (ok && col < args.n_out) {
+            if (EPI == MOE_EPI_WEIGHT_SCATTER)
+              store_row_chunk_f32(args.Cf + drow * args.ldc + col, v, scale);
+            else
+              store_row_chunk(args.C + drow * args.ldc + col, v, scale);
+          }
         }
       }
       tc_fence_before();
@@ -345,6 +359,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, G_TMEM_COLS);
   }
@@ -428,6 +443,7 @@ int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, in
   a.w_sorted = w_sorted;
   a.perm = perm;
   a.C = reinterpret_cast<__nv_bfloat16*>(C);
+  a.Cf = reinterpret_cast<float*>(C);
   a.status = status;
   a.timeout_ns = timeout_ns;
   if (epi == MOE_EPI_SWIGLU) {

@@ -59,14 +59,50 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float
   acc[7] = fmaf(wk, p3.y, acc[7]);
 }
 
+// Eight consecutive elements of a row, widened to fp32: one 16-byte load of bf16,
+// or two 16-byte loads of fp32.
+template <bool F32>
+struct Vec8;
+template <>
+struct Vec8<false> {
+  uint4 u;
+  __device__ __forceinline__ void load(const void* row, int32_t c) {
+    u = __ldg(reinterpret_cast<const uint4*>(row) + c);
+  }
+  __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void fma_into(float (&acc)[8], float wk) const { acc_bf16x8(acc, u, wk); }
+};
+template <>
+struct Vec8<true> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* row, int32_t c) {
+    const float4* p = reinterpret_cast<const float4*>(row) + 2 * c;
+    a = __ldg(p);
+    b = __ldg(p + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void fma_into(float (&acc)[8], float wk) const {
+    acc[0] = fmaf(wk, a.x, acc[0]);
+    acc[1] = fmaf(wk, a.y, acc[1]);
+    acc[2] = fmaf(wk, a.z, acc[2]);
+    acc[3] = fmaf(wk, a.w, acc[3]);
+    acc[4] = fmaf(wk, b.x, acc[4]);
+    acc[5] = fmaf(wk, b.y, acc[5]);
+    acc[6] = fmaf(wk, b.z, acc[6]);
+    acc[7] = fmaf(wk, b.w, acc[7]);
+  }
+};
+
 // out[t] = bf16(sum_k w[t,k] * y[row(t,k)]), row(t,k) = inv ? inv[t*topk+k] : t*topk+k.
-template <int KMAX>
+// y is bf16 or fp32 [R, H]; vpr = H / 8 groups of eight elements per row.
+template <int KMAX, bool F32>
 __global__ void __launch_bounds__(PM_THREADS)
-    combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
+    combine_kernel(const uint8_t* __restrict__ y, const int32_t* __restrict__ inv,
                    const float* __restrict__ w, int32_t M, int32_t R, int32_t topk,
                    int32_t vpr, uint4* __restrict__ out, int32_t* status) {
   const int lane = threadIdx.x & 31;
   const int32_t nwarps = (gridDim.x * PM_THREADS) >> 5;
+  const int64_t row_bytes = static_cast<int64_t>(vpr) * (F32 ? 32 : 16);
   for (int32_t t = (blockIdx.x * PM_THREADS + threadIdx.x) >> 5; t < M; t += nwarps) {
     int32_t my_row = 0;
     float my_w = 1.0f;
@@ -88,15 +124,18 @@ __global__ void __launch_bounds__(PM_THREADS)
     }
     uint4* dst = out + static_cast<int64_t>(t) * vpr;
     for (int32_t c = lane; c < vpr; c += 32) {
-      uint4 v[KMAX];
+      Vec8<F32> v[KMAX];
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k)
-        v[k] = (k < topk && rows[k] >= 0) ? __ldg(y + static_cast<int64_t>(rows[k]) * vpr + c)
-                                          : make_uint4(0, 0, 0, 0);
+      for (int k = 0; k < KMAX; ++k) {
+        if (k < topk && rows[k] >= 0)
+          v[k].load(y + static_cast<int64_t>(rows[k]) * row_bytes, c);
+        else
+          v[k].zero();
+      }
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < KMAX; ++k)
-        if (k < topk) acc_bf16x8(acc, v[k], wk[k]);
+        if (k < topk) v[k].fma_into(acc, wk[k]);
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
@@ -124,26 +163,36 @@ cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const void* y, const int32_t* inv, const float* w, int64_t M,
-                           int64_t H, int32_t topk, void* out, int32_t* status, int num_sms,
-                           cudaStream_t stream) {
+template <bool F32>
+static void launch_combine_t(int grid, cudaStream_t stream, const uint8_t* y, const int32_t* inv,
+                             const float* w, int32_t m, int32_t R, int32_t topk, int32_t vpr,
+                             uint4* ov, int32_t* status) {
+  if (topk <= 2)
+    combine_kernel<2, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 4)
+    combine_kernel<4, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 8)
+    combine_kernel<8, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+  else if (topk <= 16)
+    combine_kernel<16, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+  else
+    combine_kernel<32, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+}
+
+cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
+                           int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
+                           int num_sms, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   const int grid = grid_for_rows(M, num_sms);
   const int32_t R = static_cast<int32_t>(M * topk);
   const int32_t vpr = static_cast<int32_t>(H / 8);
-  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  const uint8_t* yb = reinterpret_cast<const uint8_t*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out);
   const int32_t m = static_cast<int32_t>(M);
-  if (topk <= 2)
-    combine_kernel<2><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 4)
-    combine_kernel<4><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 8)
-    combine_kernel<8><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 16)
-    combine_kernel<16><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+  if (y_f32)
+    launch_combine_t<true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
   else
-    combine_kernel<32><<<grid, PM_THREADS, 0, stream>>>(yv, inv, w, m, R, topk, vpr, ov, status);
+    launch_combine_t<false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
   return cudaGetLastError();
 }
 

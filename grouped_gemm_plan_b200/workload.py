@@ -74,6 +74,9 @@ WORKLOADS: dict[str, Workload] = {
     "wide128": Workload("wide128", 128, seed=128, **_WIDE),
     "wide512": Workload("wide512", 512, seed=512, **_WIDE),
     "wide2048": Workload("wide2048", 2048, seed=2048, **_WIDE),
+    # profiling size: the Mixtral expert shape with two experts (0.7 GB of weights,
+    # still far above L2), used for single-kernel hardware-counter captures
+    "mixtral_prof": Workload("mixtral_prof", 2048, 4096, 14336, 2, 2, "balanced", 0.0, 101),
 }
 
 

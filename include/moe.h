@@ -73,8 +73,10 @@ typedef enum moe_epilogue {
    * C is [R, N/2].  ([PTO] "MegaMoE 融合算子七阶段": SwiGLU consumes GMM1's
    * output as soon as it is produced.) */
   MOE_EPI_SWIGLU = 1,
-  /* C[perm[s], n] = bf16(w_sorted[s] * acc[s, n]): the gate-weighted row goes
-   * straight to its token-major slot i = t*topk + k; C is [R, N]. */
+  /* C[perm[s], n] = w_sorted[s] * acc[s, n]: the gate-weighted row goes straight
+   * to its token-major slot i = t*topk + k; C is FP32 [R, N].  It stays in fp32
+   * because moe_combine sums it once more: one bf16 rounding fewer on the path
+   * to the layer output. */
   MOE_EPI_WEIGHT_SCATTER = 2
 } moe_epilogue;
 
@@ -152,11 +154,13 @@ moe_status moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets
  *               t*topk + k           if inv_perm == NULL (y token-major, as
  *                                    written by MOE_EPI_WEIGHT_SCATTER)
  *   wk = topk_w[t*topk + k] if topk_w != NULL, else 1.
- *   y bf16 [R, H], out bf16 [M, H]; H a multiple of 8.
+ *   y [R, H] is bf16 (y_fp32 = 0) or fp32 (y_fp32 = 1); out bf16 [M, H];
+ *   H a multiple of 8.  An index outside [0, R) contributes zero and records
+ *   MOE_ERR_BAD_INDEX.
  */
-moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk_w, int64_t M,
-                       int64_t H, int32_t topk, void* out, void* ws, size_t ws_bytes,
-                       void* stream);
+moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
+                       const float* topk_w, int64_t M, int64_t H, int32_t topk, void* out,
+                       void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_ffn_fused -- the whole layer:
@@ -165,9 +169,9 @@ moe_status moe_combine(const void* y, const int32_t* inv_perm, const float* topk
  *   x bf16 [M, H], W1 bf16 [E, H, 2F], W2 bf16 [E, F, H], out bf16 [M, H].
  * It runs plan -> dispatch -> GEMM1 with the SwiGLU epilogue -> GEMM2 with the
  * gate-weight scatter epilogue -> combine.  counts [E], offsets [E+1] and perm
- * [R] receive the plan (as moe_plan).  The intermediates (expert-ordered x, the
- * SwiGLU activations, the weighted expert outputs) live in the workspace
- * (moe_workspace_size(MOE_OP_FFN_FUSED, ...)).
+ * [R] receive the plan (as moe_plan).  The intermediates (expert-ordered x and
+ * the SwiGLU activations in bf16, the gate-weighted expert outputs in fp32)
+ * live in the workspace (moe_workspace_size(MOE_OP_FFN_FUSED, ...)).
  *   n_c: thread blocks given to the memory stages (dispatch / combine) while the
  *   GEMM blocks run, [COMET] 4.2.2.  0 runs the stages as consecutive kernels;
  *   -1 takes the value from the library's profiled table for this shape.

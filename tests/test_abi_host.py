@@ -45,7 +45,7 @@ def test_workspace_sizes(lib):
         assert B.moe_workspace_size(op, 4096, 4096, 14336, 8, 2) == 256
     R, H, F = 8192, 4096, 14336
     fused = B.moe_workspace_size(B.OP_FFN_FUSED, 4096, H, F, 8, 2)
-    assert fused >= 256 + 2 * R * H * 2 + R * F * 2 + R * 4
+    assert fused >= 256 + R * H * 2 + R * F * 2 + R * H * 4 + R * 4
     assert B.moe_workspace_size(B.OP_FFN_FUSED, 0, H, F, 8, 2) == 256
 
 
@@ -100,11 +100,12 @@ def test_dispatch_combine_validation(lib):
     assert lib.moe_dispatch(FAKE, FAKE, 4, 64, 0, FAKE, FAKE_WS, 256, None) == 1    # topk
     assert lib.moe_dispatch(ctypes.c_void_p(0x10004), FAKE, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 7
     assert lib.moe_dispatch(None, FAKE, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 1
-    assert lib.moe_combine(FAKE, FAKE, FAKE, 4, 64, 2, None, FAKE_WS, 256, None) == 1
-    assert lib.moe_combine(FAKE, FAKE, FAKE, 4, 64, 33, FAKE, FAKE_WS, 256, None) == 1
+    assert lib.moe_combine(FAKE, 0, FAKE, FAKE, 4, 64, 2, None, FAKE_WS, 256, None) == 1
+    assert lib.moe_combine(FAKE, 0, FAKE, FAKE, 4, 64, 33, FAKE, FAKE_WS, 256, None) == 1
+    assert lib.moe_combine(FAKE, 2, FAKE, FAKE, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 1
     # M = 0 is a no-op even with null data pointers
     assert lib.moe_dispatch(None, None, 0, 64, 2, None, FAKE_WS, 256, None) == 0
-    assert lib.moe_combine(None, None, None, 0, 64, 2, None, FAKE_WS, 256, None) == 0
+    assert lib.moe_combine(None, 0, None, None, 0, 64, 2, None, FAKE_WS, 256, None) == 0
 
 
 def test_fused_validation(lib):

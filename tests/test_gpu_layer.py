@@ -5,7 +5,11 @@ Small and medium shapes are compared element by element with the full oracle.
 The five workload shapes are run at full size in the launch configuration the
 benchmark times; there the plan is compared bit for bit, a sample of output rows
 is compared with the oracle's per-token brute force, and the fused output is
-compared with the chain of separate calls over every element."""
+compared with the chain of separate calls over every element.
+
+Bar (the benchmark spec tolerance, read for a bf16 output): relative Frobenius <= 1e-2
+and per element |err| <= 2e-2 * rms(ref) + half a bf16 ulp of ref per bf16
+rounding on the path after the last GEMM (see helpers.check_close)."""
 import numpy as np
 import pytest
 import torch
@@ -87,7 +91,8 @@ def test_layer_matches_oracle(cuda_dev, M, H, F, E, topk, kind):
     assert np.array_equal(offsets.cpu().numpy(), ro)
     assert np.array_equal(perm.cpu().numpy(), rp)
     chain = run_chain(cuda_dev, x, W1, W2, ids, tw)
-    check_close(chain, ref, "chain of calls")
+    # the chain stores the expert outputs in bf16 before combining: one rounding more
+    check_close(chain, ref, "chain of calls", ulps=2.0)
 
 
 def test_layer_empty_batch(cuda_dev):
@@ -157,4 +162,8 @@ def test_workload_full_size(cuda_dev, name):
     ref_rows = oracle.bruteforce_tokens(x, W1c, W2c, ids, tw, tokens)
     check_close(out.cpu()[torch.from_numpy(tokens)], ref_rows, f"{name} sampled rows")
     chain = run_chain(cuda_dev, x, W1, W2, ids, tw)
-    check_close(out, chain.double().cpu().numpy(), f"{name} fused vs chain")
+    chain_rows = chain.cpu()[torch.from_numpy(tokens)]
+    check_close(chain_rows, ref_rows, f"{name} chain sampled rows", ulps=2.0)
+    # two bf16 results of the same layer: within the bar of each other, one
+    # rounding of each allowed
+    check_close(out, chain.double().cpu().numpy(), f"{name} fused vs chain", ulps=3.0)

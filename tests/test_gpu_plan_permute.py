@@ -128,14 +128,15 @@ def test_dispatch_bad_index(cuda_dev):
     assert bool((xp[3] == 0).all())
 
 
-@pytest.mark.parametrize("M,H,E,topk,token_major", [(256, 256, 8, 2, False), (333, 2048, 64, 4, False),
-                                                    (64, 7168, 16, 8, True), (1000, 4096, 16, 2, True),
-                                                    (9, 64, 40, 32, False)])
-def test_combine(cuda_dev, M, H, E, topk, token_major):
+@pytest.mark.parametrize("M,H,E,topk,token_major,ydt", [
+    (256, 256, 8, 2, False, torch.bfloat16), (333, 2048, 64, 4, False, torch.bfloat16),
+    (64, 7168, 16, 8, True, torch.float32), (1000, 4096, 16, 2, True, torch.float32),
+    (9, 64, 40, 32, False, torch.float32), (50, 128, 8, 3, True, torch.bfloat16)])
+def test_combine(cuda_dev, M, H, E, topk, token_major, ydt):
     ids, w = routing_case(M, E, topk, "uniform", seed=M)
     _, _, perm, inv, _ = oracle.plan(ids, w, E)
     R = M * topk
-    y = torch.randn(R, H).to(torch.bfloat16)
+    y = torch.randn(R, H).to(ydt)
     yd = y.double().numpy()
     out, check = guarded_empty((M, H), torch.bfloat16, cuda_dev)
     ws = B.alloc_workspace(B.OP_COMBINE, M, H, 0, E, topk, cuda_dev)
