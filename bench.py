@@ -344,11 +344,15 @@ def run_ours(args):
     flops_g1 = 4.0 * R * H * F
     g1_s = stage_avg["gemm1_swiglu"] / 1e3
     achieved = flops_g1 / g1_s / 1e12
-    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    # The timed region is short (tens of ms of GPU work between L2 flushes) and the
+    # sampled SM clock stays near its maximum, so the kernel is held to the burst
+    # figure of the measured cuBLAS bf16 GEMM, not to the power-capped sustained one.
+    peak = pk["bf16_tflops"]
     traffic = measured_traffic("gemm1_swiglu", wl.name)
     roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{pk_kind} bf16_tflops_sustained", "traffic": traffic,
+                "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                "peak_sustained": pk.get("bf16_tflops_sustained"), "traffic": traffic,
                 "algorithmic": f"4*R*H*F = {flops_g1:.4g} FLOP per launch"}
     g2 = 2.0 * R * H * F / (stage_avg["gemm2_scatter"] / 1e3) / 1e12
     disp_bytes = M * H * 2 + R * H * 2 + R * 4
