@@ -28,8 +28,8 @@ OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED = 0, 1, 2, 3, 4
 
 # Every symbol include/moe.h declares.
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_plan", "moe_dispatch",
-           "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_get_device_status",
-           "moe_set_wait_timeout_ns", "moe_last_error"]
+           "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
+           "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_last_error"]
 
 
 class MoEError(RuntimeError):
@@ -70,6 +70,8 @@ def load(path: str | None = None):
     lib.moe_combine.restype = st
     lib.moe_ffn_fused.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]
     lib.moe_ffn_fused.restype = st
+    lib.moe_ffn_fused_noalloc.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P, P]
+    lib.moe_ffn_fused_noalloc.restype = st
     lib.moe_get_device_status.argtypes = [P, P]
     lib.moe_get_device_status.restype = st
     lib.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
@@ -155,6 +157,17 @@ def moe_ffn_fused(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, ws, n
     _check(load().moe_ffn_fused(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w), M, H,
                                 F2 // 2, E, topk, n_c, _ptr(out), _ptr(counts), _ptr(offsets),
                                 _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_ffn_fused_noalloc(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, status=None,
+                          stream=None):
+    """The layer without a workspace: intermediates in the library's own device scratch."""
+    M, H = x.shape
+    E, _, F2 = W1.shape
+    topk = topk_ids.shape[1]
+    _check(load().moe_ffn_fused_noalloc(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w),
+                                        M, H, F2 // 2, E, topk, _ptr(out), _ptr(counts),
+                                        _ptr(offsets), _ptr(perm), _ptr(status), _stream(stream)))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

@@ -114,6 +114,15 @@ moe_status check_route(int64_t M, int32_t E, int32_t topk) {
 
 }  // namespace
 
+namespace moe {
+// Used by entry points defined in other files of the library.
+moe_status record_error(moe_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+uint64_t wait_timeout_ns() { return g_timeout_ns; }
+}  // namespace moe
+
 extern "C" {
 
 int moe_abi_version(void) { return 1; }

@@ -183,6 +183,45 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
                          int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* Size of the library's own device scratch used by moe_ffn_fused_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * moe_ffn_fused_noalloc -- the same layer as moe_ffn_fused, for callers that
+ * cannot allocate device memory.  The pages have no counterpart of this call.
+ *
+ * Who needs it: a host program that is handed only its input and output
+ * buffers (a C or plugin caller with no device allocator of its own), or a
+ * process whose device memory was reserved up front by another allocator, has
+ * no way to provide the workspace moe_ffn_fused asks for -- a cudaMalloc would
+ * fail, or would stall the device at a bad moment.  This call takes no
+ * workspace and allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library routine).  Its intermediates live in a fixed device array of
+ * MOE_NOALLOC_SCRATCH_BYTES (64 MiB) inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * Arguments are those of moe_ffn_fused without n_c and workspace (the stages
+ * run as consecutive kernels on `stream`), plus
+ *   status  int32 [1] device pointer (may be NULL): receives this call's device
+ *           status word (a moe_status; MOE_ERR_BAD_EXPERT_ID etc.).
+ * Limit: the intermediates of R = M*topk rows need
+ *   256 + R*H*2 + R*F*2 + R*H*4 + R*4 bytes (each part rounded up to 256);
+ * a shape that needs more than MOE_NOALLOC_SCRATCH_BYTES is rejected with
+ * MOE_ERR_WORKSPACE_TOO_SMALL before anything is launched (e.g. H=7168, F=4096,
+ * topk=8 fits up to M=163 tokens; H=4096, F=14336, topk=2 up to M=630).
+ * The first call on a device looks up the array's device address (with that
+ * device current) and remembers it; make that first call before any stream
+ * capture.  Every call shares the one array and it keeps the previous call's
+ * contents: calls that overlap on the GPU (on different streams, or from
+ * different threads without ordering) race on it and must be serialised by the
+ * caller.
+ */
+moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const void* W2,
+                                 const int32_t* topk_ids, const float* topk_w, int64_t M,
+                                 int64_t H, int64_t F, int32_t E, int32_t topk, void* out,
+                                 int32_t* counts, int32_t* offsets, int32_t* perm,
+                                 int32_t* status, void* stream);
+
 /* Synchronises `stream`, returns the device status word of `ws` (a moe_status)
  * and clears it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error. */
 moe_status moe_get_device_status(void* ws, void* stream);
