@@ -29,7 +29,8 @@ OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED = 0, 1, 2, 3, 4
 # Every symbol include/moe.h declares.
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_plan", "moe_dispatch",
            "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
-           "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_last_error"]
+           "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
+           "moe_last_error"]
 
 
 class MoEError(RuntimeError):
@@ -76,6 +77,8 @@ def load(path: str | None = None):
     lib.moe_get_device_status.restype = st
     lib.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.moe_set_wait_timeout_ns.restype = None
+    lib.moe_set_fault_injection.argtypes = [i32, i32]
+    lib.moe_set_fault_injection.restype = st
     lib.moe_last_error.restype = ctypes.c_char_p
     if path is None:
         _lib = lib
@@ -177,6 +180,11 @@ def moe_get_device_status(ws, stream=None) -> int:
 
 def moe_set_wait_timeout_ns(ns: int) -> None:
     load().moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_set_fault_injection(kind: int, index: int = 0) -> None:
+    """Test hook (see include/moe.h): 1 = withhold one m-tile's dispatch flag, 0 = off."""
+    _check(load().moe_set_fault_injection(int(kind), int(index)))
 
 
 def moe_last_error() -> str:

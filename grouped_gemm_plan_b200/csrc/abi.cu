@@ -14,7 +14,7 @@
 namespace moe {
 cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
-                        int32_t* status, int num_sms, cudaStream_t stream);
+                        int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
@@ -24,12 +24,20 @@ int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, in
                         int64_t R, int64_t K, int64_t N, int epi, const float* w_sorted,
                         const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                         int num_sms, cudaStream_t stream);
+size_t layer_sync_bytes(int64_t M, int64_t R, int32_t E);
+int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_t* perm,
+                     const float* w_sorted, const int32_t* offsets, void* xp, void* h, void* yk,
+                     void* out, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk,
+                     int32_t n_c, int32_t* status, void* sync_area, uint64_t timeout_ns,
+                     int32_t withhold_mtile, int num_sms, cudaStream_t stream);
+int32_t profiled_n_c(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
 }  // namespace moe
 
 namespace {
 
 thread_local std::string g_last_error;
 uint64_t g_timeout_ns = 2000000000ull;
+int32_t g_withhold_mtile = -1;  // fault injection for tests (moe_set_fault_injection)
 
 constexpr size_t kCtrlBytes = 256;
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
@@ -69,15 +77,22 @@ int num_sms_current() {
 
 int32_t* status_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 
+// Per-chunk histograms of the plan: up to 256 chunks of E + 1 ints.
+size_t plan_scratch_bytes(int32_t E) { return align256(size_t(256) * size_t(E + 1) * 4); }
+
+int32_t* plan_scratch(void* ws) {
+  return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kCtrlBytes);
+}
+
 // Intermediates of moe_ffn_fused inside the workspace.
 struct FusedLayout {
-  size_t xp, h, yk, w_sorted, total;
+  size_t xp, h, yk, w_sorted, sync, total;
 };
 
-FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t topk) {
+FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
   const int64_t R = M * topk;
   FusedLayout L;
-  size_t off = kCtrlBytes;
+  size_t off = kCtrlBytes + plan_scratch_bytes(E);
   L.xp = off;
   off += align256(size_t(R) * size_t(H) * 2);
   L.h = off;
@@ -86,6 +101,8 @@ FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t topk) {
   off += align256(size_t(R) * size_t(H) * 4);
   L.w_sorted = off;
   off += align256(size_t(R) * 4);
+  L.sync = off;  // flags and counters of the single-kernel layer
+  off += align256(moe::layer_sync_bytes(M, R, E));
   L.total = off;
   return L;
 }
@@ -131,10 +148,22 @@ const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns > 0 ? ns : 1; }
 
+moe_status moe_set_fault_injection(int32_t kind, int32_t index) {
+  if (kind == 0) {
+    g_withhold_mtile = -1;
+    return MOE_OK;
+  }
+  if (kind == 1 && index >= 0) {
+    g_withhold_mtile = index;
+    return MOE_OK;
+  }
+  return fail(MOE_ERR_INVALID_ARG, "unknown fault injection kind %d", kind);
+}
+
 size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
-  (void)E;
-  if (M < 0 || H < 0 || F < 0 || topk < 0) return kCtrlBytes;
-  if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, topk).total;
+  if (M < 0 || H < 0 || F < 0 || topk < 0 || E < 1 || E > MOE_MAX_EXPERTS) return kCtrlBytes;
+  if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, E, topk).total;
+  if (op == MOE_OP_PLAN) return kCtrlBytes + plan_scratch_bytes(E);
   return kCtrlBytes;
 }
 
@@ -165,7 +194,8 @@ moe_status moe_plan(const int32_t* topk_ids, const float* topk_w, int64_t M, int
   if (st != MOE_OK) return st;
   cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(M * topk), E, counts,
                                      offsets, perm, inv_perm, w_sorted, status_word(ws),
-                                     num_sms_current(), reinterpret_cast<cudaStream_t>(stream));
+                                     plan_scratch(ws), num_sms_current(),
+                                     reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "moe_plan launch");
   return MOE_OK;
 }
@@ -259,7 +289,8 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     // Still a defined plan: zero counts and offsets.
     cudaStream_t s0 = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err = moe::launch_plan(topk_ids, topk_w, 0, E, counts, offsets, perm, nullptr,
-                                       nullptr, status_word(ws), num_sms_current(), s0);
+                                       nullptr, status_word(ws), plan_scratch(ws),
+                                       num_sms_current(), s0);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ffn_fused plan");
   }
   if (x == nullptr || W1 == nullptr || W2 == nullptr || topk_ids == nullptr || topk_w == nullptr ||
@@ -269,7 +300,7 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     return fail(MOE_ERR_MISALIGNED, "x, W1, W2 and out must be 16-byte aligned");
 
   const int64_t R = M * topk;
-  const FusedLayout L = fused_layout(M, H, F, topk);
+  const FusedLayout L = fused_layout(M, H, F, E, topk);
   uint8_t* base = static_cast<uint8_t*>(ws);
   void* xp = base + L.xp;
   void* h = base + L.h;
@@ -280,8 +311,20 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
-                                     perm, nullptr, w_sorted, status, sms, s);
+                                     perm, nullptr, w_sorted, status, plan_scratch(ws), sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused plan");
+  const int32_t nc = n_c < 0 ? moe::profiled_n_c(M, H, F, E, topk) : n_c;
+  if (nc > 0) {
+    // One persistent kernel: nc memory CTAs (dispatch, combine) beside the GEMM CTAs.
+    if (nc > 64 || nc >= sms) return fail(MOE_ERR_INVALID_ARG, "n_c = %d must be < min(65, #SMs = %d)", nc, sms);
+    const int rc = moe::launch_moe_layer(x, W1, W2, perm, w_sorted, offsets, xp, h, yk, out, M, H, F,
+                                         E, topk, nc, status, base + L.sync, g_timeout_ns,
+                                         g_withhold_mtile, sms, s);
+    if (rc == 1) return fail(MOE_ERR_CUDA, "tensor map encode failed (layer kernel)");
+    if (rc == 3) return fail(MOE_ERR_CUDA, "cooperative launch refused: the layer kernel needs one co-resident CTA per SM");
+    if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_ffn_fused layer kernel");
+    return MOE_OK;
+  }
   err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused dispatch");
   int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,

@@ -22,7 +22,7 @@
 namespace moe {
 cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
-                        int32_t* status, int num_sms, cudaStream_t stream);
+                        int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
@@ -51,14 +51,16 @@ int g_num_sms[kMaxDevices] = {0};
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t xp, h, yk, w_sorted, total;
+  size_t hist, xp, h, yk, w_sorted, total;
 };
 
-// status word [0, 256), then xp bf16 [R, H], h bf16 [R, F], yk fp32 [R, H],
-// w_sorted fp32 [R]
-Layout layout(int64_t R, int64_t H, int64_t F) {
+// status word [0, 256), the plan's per-chunk histograms (256 x (E + 1) int32),
+// then xp bf16 [R, H], h bf16 [R, F], yk fp32 [R, H], w_sorted fp32 [R]
+Layout layout(int64_t R, int64_t H, int64_t F, int32_t E) {
   Layout L;
   size_t off = 256;
+  L.hist = off;
+  off += al256(size_t(256) * size_t(E + 1) * 4);
   L.xp = off;
   off += al256(size_t(R) * size_t(H) * 2);
   L.h = off;
@@ -111,7 +113,7 @@ extern "C" moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const
   if (H > (int64_t(1) << 30) || F > (int64_t(1) << 29))
     return record_error(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
   const int64_t R = M * topk;
-  const Layout L = layout(R, H, F);
+  const Layout L = layout(R, H, F, E);
   if (L.total > size_t(MOE_NOALLOC_SCRATCH_BYTES))
     return record_error(MOE_ERR_WORKSPACE_TOO_SMALL,
                         "this shape needs " + std::to_string(L.total) +
@@ -141,7 +143,8 @@ extern "C" moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const
   err = cudaMemsetAsync(st, 0, sizeof(int32_t), s);
   if (err == cudaSuccess)
     err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets, perm,
-                           nullptr, reinterpret_cast<float*>(b + L.w_sorted), st, sms, s);
+                           nullptr, reinterpret_cast<float*>(b + L.w_sorted), st,
+                           reinterpret_cast<int32_t*>(b + L.hist), sms, s);
   if (err == cudaSuccess && R > 0)
     err = moe::launch_dispatch(x, perm, M, H, topk, b + L.xp, st, sms, s);
   if (err != cudaSuccess)

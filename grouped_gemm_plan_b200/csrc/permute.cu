@@ -7,42 +7,41 @@
 // Combine is the top-k weighted accumulation ("MoE dispatch/combine 为什么慢":
 // topK 加权累加) plus Unpermute.
 //
-// Layout of the work: one warp per output row; each lane moves 16-byte vectors
-// (8 bf16), 32 lanes cover 512 contiguous bytes per step, so every access is a
-// full, coalesced 128-byte line.  Grids are a multiple of the SM count with 8
-// warps per CTA; rows are walked grid-stride.  Combine reads the top-k source
-// vectors of a step before it accumulates, so up to topk loads per lane are in
-// flight; the sum runs in fp32 registers in ascending k, one bf16 cast at the end.
+// Layout of the work: a work item is one 512-byte step of one output row, done by
+// one warp; each lane moves a 16-byte vector (8 bf16), so every access is a full,
+// coalesced 128-byte line, and even a batch of a few rows spreads over all SMs.
+// Grids are a multiple of the SM count with 8 warps per CTA; items are walked
+// grid-stride.  Combine reads the top-k source vectors of a step before it
+// accumulates, so up to topk loads per lane are in flight; the sum runs in fp32
+// registers in ascending k, one bf16 cast at the end.
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int PM_THREADS = 256;
 
+// Work item = (row s, step q): lane l of the warp copies 16-byte vector
+// q*32 + l of the row.  Splitting rows into 512-byte steps keeps every SM busy
+// even when there are only a few rows (small batches).
 __global__ void __launch_bounds__(PM_THREADS)
     dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int32_t R,
                     int32_t topk, int32_t vpr, uint4* __restrict__ xp, int32_t* status) {
   const int lane = threadIdx.x & 31;
-  const int32_t nwarps = (gridDim.x * PM_THREADS) >> 5;
-  for (int32_t s = (blockIdx.x * PM_THREADS + threadIdx.x) >> 5; s < R; s += nwarps) {
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
+  const int32_t steps = (vpr + 31) >> 5;
+  const int64_t items = static_cast<int64_t>(R) * steps;
+  for (int64_t it = (static_cast<int64_t>(blockIdx.x) * PM_THREADS + threadIdx.x) >> 5; it < items;
+       it += nwarps) {
+    const int32_t s = static_cast<int32_t>(it / steps);
+    const int32_t c = static_cast<int32_t>(it - static_cast<int64_t>(s) * steps) * 32 + lane;
     const int32_t i = __ldg(perm + s);
     uint4* dst = xp + static_cast<int64_t>(s) * vpr;
     if (i < 0 || i >= R) {
       if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
-      for (int32_t c = lane; c < vpr; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+      if (c < vpr) dst[c] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    const uint4* src = x + static_cast<int64_t>(i / topk) * vpr;
-    int32_t c = lane;
-    for (; c + 96 < vpr; c += 128) {
-      const uint4 a0 = __ldg(src + c), a1 = __ldg(src + c + 32), a2 = __ldg(src + c + 64),
-                  a3 = __ldg(src + c + 96);
-      dst[c] = a0;
-      dst[c + 32] = a1;
-      dst[c + 64] = a2;
-      dst[c + 96] = a3;
-    }
-    for (; c < vpr; c += 32) dst[c] = __ldg(src + c);
+    if (c < vpr) dst[c] = __ldg(x + static_cast<int64_t>(i / topk) * vpr + c);
   }
 }
 
@@ -101,9 +100,15 @@ __global__ void __launch_bounds__(PM_THREADS)
                    const float* __restrict__ w, int32_t M, int32_t R, int32_t topk,
                    int32_t vpr, uint4* __restrict__ out, int32_t* status) {
   const int lane = threadIdx.x & 31;
-  const int32_t nwarps = (gridDim.x * PM_THREADS) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
   const int64_t row_bytes = static_cast<int64_t>(vpr) * (F32 ? 32 : 16);
-  for (int32_t t = (blockIdx.x * PM_THREADS + threadIdx.x) >> 5; t < M; t += nwarps) {
+  const int32_t steps = (vpr + 31) >> 5;
+  const int64_t items = static_cast<int64_t>(M) * steps;
+  // Work item = (token t, step q): lane l handles group q*32 + l of eight elements.
+  for (int64_t it = (static_cast<int64_t>(blockIdx.x) * PM_THREADS + threadIdx.x) >> 5; it < items;
+       it += nwarps) {
+    const int32_t t = static_cast<int32_t>(it / steps);
+    const int32_t c = static_cast<int32_t>(it - static_cast<int64_t>(t) * steps) * 32 + lane;
     int32_t my_row = 0;
     float my_w = 1.0f;
     if (lane < topk) {
@@ -122,33 +127,32 @@ __global__ void __launch_bounds__(PM_THREADS)
       rows[k] = __shfl_sync(0xffffffffu, my_row, k);
       wk[k] = __shfl_sync(0xffffffffu, my_w, k);
     }
-    uint4* dst = out + static_cast<int64_t>(t) * vpr;
-    for (int32_t c = lane; c < vpr; c += 32) {
-      Vec8<F32> v[KMAX];
+    if (c >= vpr) continue;
+    Vec8<F32> v[KMAX];
 #pragma unroll
-      for (int k = 0; k < KMAX; ++k) {
-        if (k < topk && rows[k] >= 0)
-          v[k].load(y + static_cast<int64_t>(rows[k]) * row_bytes, c);
-        else
-          v[k].zero();
-      }
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < KMAX; ++k)
-        if (k < topk) v[k].fma_into(acc, wk[k]);
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      dst[c] = o;
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < topk && rows[k] >= 0)
+        v[k].load(y + static_cast<int64_t>(rows[k]) * row_bytes, c);
+      else
+        v[k].zero();
     }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+      if (k < topk) v[k].fma_into(acc, wk[k]);
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    out[static_cast<int64_t>(t) * vpr + c] = o;
   }
 }
 
-static int grid_for_rows(int64_t rows, int num_sms) {
+// Grid for `items` warp-sized work items: up to 8 CTAs of 8 warps per SM.
+static int grid_for_items(int64_t items, int num_sms) {
   const int64_t per_cta = PM_THREADS / 32;
-  const int64_t want = (rows + per_cta - 1) / per_cta;
+  const int64_t want = (items + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
 }
@@ -157,7 +161,8 @@ cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream) {
   const int64_t R = M * topk;
   if (R == 0) return cudaSuccess;
-  dispatch_kernel<<<grid_for_rows(R, num_sms), PM_THREADS, 0, stream>>>(
+  const int64_t steps = (H / 8 + 31) / 32;
+  dispatch_kernel<<<grid_for_items(R * steps, num_sms), PM_THREADS, 0, stream>>>(
       reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
       static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
   return cudaGetLastError();
@@ -183,7 +188,7 @@ cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const 
                            int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
                            int num_sms, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
-  const int grid = grid_for_rows(M, num_sms);
+  const int grid = grid_for_items(M * ((H / 8 + 31) / 32), num_sms);
   const int32_t R = static_cast<int32_t>(M * topk);
   const int32_t vpr = static_cast<int32_t>(H / 8);
   const uint8_t* yb = reinterpret_cast<const uint8_t*>(y);

@@ -7,16 +7,21 @@
 //   offsets    = exclusive prefix sum of counts (E+1 entries)
 //   perm[s]    = i for the slots s of expert e, in ascending i (stable)
 //
-// One launch.  The R routed rows are cut into chunks, one CTA per chunk.  Every
-// CTA reads the whole id array (R int32, served from L2) to build the total
-// histogram and the histogram of the rows before its chunk -- warp-aggregated
-// with __match_any_sync so that a popular expert costs one shared atomic per
-// warp, not one per lane.  A block scan turns the totals into offsets.  Then the
-// CTA ranks its own rows: warp w owns a contiguous segment of the chunk, counts
-// it per expert, the per-warp counts are scanned in warp order, and a second
-// pass over the segment gives every row its slot = offsets[e] + rows of e before
-// the chunk + rows of e in earlier warps + rows of e earlier in this warp.
-// Stability holds by construction: slots grow with i.
+// Two launches when the rows span several chunks (one CTA per chunk), one when
+// they fit a single chunk:
+//   plan_hist_kernel   each CTA histograms its own chunk (warp-aggregated with
+//                      __match_any_sync, so a popular expert costs one shared
+//                      atomic per warp) and writes it, plus its count of invalid
+//                      ids, to a per-chunk row of the workspace scratch;
+//   plan_kernel        each CTA sums the chunk rows into the totals and the rows
+//                      of each expert in earlier chunks, scans the totals into
+//                      offsets, then ranks its own rows: warp w owns a contiguous
+//                      segment of the chunk, counts it per expert, the per-warp
+//                      counts are scanned in warp order, and a second pass gives
+//                      every row its slot = offsets[e] + rows of e in earlier
+//                      chunks + rows of e in earlier warps + rows of e earlier in
+//                      this warp.  Stability holds by construction: slots grow
+//                      with i.
 #include "common.cuh"
 
 namespace moe {
@@ -24,12 +29,42 @@ namespace moe {
 constexpr int PLAN_THREADS = 512;
 constexpr int PLAN_WARPS = PLAN_THREADS / 32;
 constexpr int PLAN_UNROLL = 4;
+constexpr int PLAN_MAX_CHUNKS = 256;   // rows of the per-chunk histogram scratch
+
+// Row c of `hist` (E + 1 ints): rows of each expert in chunk c, then the number
+// of ids outside [0, E) in it.
+__global__ void __launch_bounds__(PLAN_THREADS)
+    plan_hist_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t seg,
+                     int32_t* __restrict__ hist) {
+  extern __shared__ int32_t hist_smem[];  // [E]
+  __shared__ int32_t s_bad;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int32_t chunk = PLAN_WARPS * seg;
+  const int32_t c0 = blockIdx.x * chunk;
+  const int32_t c1 = min(c0 + chunk, R);
+  for (int e = tid; e < E; e += PLAN_THREADS) hist_smem[e] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int32_t base = c0; base < c1; base += PLAN_THREADS) {
+    const int32_t i = base + tid;
+    const int32_t e = i < c1 ? __ldg(ids + i) : -1;
+    const bool good = i < c1 && e >= 0 && e < E;
+    if (i < c1 && !good) atomicAdd(&s_bad, 1);
+    const unsigned peers = __match_any_sync(0xffffffffu, good ? e : -1);
+    if (good && lane == __ffs(peers) - 1) atomicAdd(&hist_smem[e], __popc(peers));
+  }
+  __syncthreads();
+  int32_t* row = hist + static_cast<int64_t>(blockIdx.x) * (E + 1);
+  for (int e = tid; e < E; e += PLAN_THREADS) row[e] = hist_smem[e];
+  if (tid == 0) row[E] = s_bad;
+}
 
 __global__ void __launch_bounds__(PLAN_THREADS)
     plan_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w, int32_t R,
-                int32_t E, int32_t seg, int32_t* __restrict__ counts,
-                int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-                int32_t* __restrict__ inv, float* __restrict__ w_sorted, int32_t* status) {
+                int32_t E, int32_t seg, const int32_t* __restrict__ hist, int32_t nchunks,
+                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                float* __restrict__ w_sorted, int32_t* status) {
   extern __shared__ int32_t plan_smem[];
   int32_t* tot = plan_smem;           // [E] totals, later exclusive offsets
   int32_t* before = plan_smem + E;    // [E] rows of e before this chunk
@@ -50,27 +85,36 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   if (tid == 0) s_bad = 0;
   __syncthreads();
 
-  // ---- pass over all rows: totals and rows before this chunk
-  for (int32_t base = 0; base < R; base += PLAN_THREADS * PLAN_UNROLL) {
-    int32_t ev[PLAN_UNROLL];
-#pragma unroll
-    for (int u = 0; u < PLAN_UNROLL; ++u) {
-      const int32_t i = base + u * PLAN_THREADS + tid;
-      ev[u] = i < R ? __ldg(ids + i) : -1;
+  if (hist != nullptr) {
+    // ---- totals and rows before this chunk, from the per-chunk histograms
+    for (int32_t idx = tid; idx < nchunks * E; idx += PLAN_THREADS) {
+      const int32_t c = idx / E, e = idx - c * E;
+      const int32_t v = hist[static_cast<int64_t>(c) * (E + 1) + e];
+      if (v != 0) {
+        atomicAdd(&tot[e], v);
+        if (c < static_cast<int32_t>(blockIdx.x)) atomicAdd(&before[e], v);
+      }
     }
+    for (int32_t c = tid; c < nchunks; c += PLAN_THREADS)
+      if (hist[static_cast<int64_t>(c) * (E + 1) + E] != 0) s_bad = 1;
+  } else {
+    // ---- a single chunk: histogram of all rows here
+    for (int32_t base = 0; base < R; base += PLAN_THREADS * PLAN_UNROLL) {
+      int32_t ev[PLAN_UNROLL];
 #pragma unroll
-    for (int u = 0; u < PLAN_UNROLL; ++u) {
-      const int32_t i = base + u * PLAN_THREADS + tid;
-      const int32_t e = ev[u];
-      const bool valid = i < R;
-      const bool good = valid && e >= 0 && e < E;
-      if (valid && !good) s_bad = 1;
-      const int32_t key = good ? (e * 2 + (i < c0 ? 1 : 0)) : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      if (good && lane == __ffs(peers) - 1) {
-        const int n = __popc(peers);
-        atomicAdd(&tot[e], n);
-        if (i < c0) atomicAdd(&before[e], n);
+      for (int u = 0; u < PLAN_UNROLL; ++u) {
+        const int32_t i = base + u * PLAN_THREADS + tid;
+        ev[u] = i < R ? __ldg(ids + i) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < PLAN_UNROLL; ++u) {
+        const int32_t i = base + u * PLAN_THREADS + tid;
+        const int32_t e = ev[u];
+        const bool valid = i < R;
+        const bool good = valid && e >= 0 && e < E;
+        if (valid && !good) s_bad = 1;
+        const unsigned peers = __match_any_sync(0xffffffffu, good ? e : -1);
+        if (good && lane == __ffs(peers) - 1) atomicAdd(&tot[e], __popc(peers));
       }
     }
   }
@@ -168,10 +212,11 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   }
 }
 
-// Host launcher (no validation here; the C ABI layer validates).
+// Host launcher (no validation here; the C ABI layer validates).  `scratch`
+// holds plan_hist_rows(E) ints (the per-chunk histograms).
 cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
-                        int32_t* status, int num_sms, cudaStream_t stream) {
+                        int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream) {
   const size_t smem = sizeof(int32_t) * (size_t)(2 + PLAN_WARPS) * (size_t)E;
   static int attr_done_mask = 0;  // one bit per device ordinal (< 31)
   int dev = 0;
@@ -185,18 +230,25 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
   }
   if (R == 0) {
     // Only counts/offsets to write: one CTA with no rows.
-    plan_kernel<<<1, PLAN_THREADS, smem, stream>>>(ids, w, 0, E, 32, counts, offsets, perm, inv,
-                                                   w_sorted, status);
+    plan_kernel<<<1, PLAN_THREADS, smem, stream>>>(ids, w, 0, E, 32, nullptr, 0, counts, offsets,
+                                                   perm, inv, w_sorted, status);
     return cudaGetLastError();
   }
-  int32_t per_cta = (R + num_sms - 1) / num_sms;
+  const int max_chunks = num_sms < PLAN_MAX_CHUNKS ? num_sms : PLAN_MAX_CHUNKS;
+  int32_t per_cta = (R + max_chunks - 1) / max_chunks;
   int32_t seg = (per_cta + PLAN_WARPS - 1) / PLAN_WARPS;
   seg = ((seg + 31) / 32) * 32;
   if (seg < 32) seg = 32;
   const int32_t chunk = seg * PLAN_WARPS;
   const int32_t grid = (R + chunk - 1) / chunk;
-  plan_kernel<<<grid, PLAN_THREADS, smem, stream>>>(ids, w, R, E, seg, counts, offsets, perm, inv,
-                                                    w_sorted, status);
+  if (grid == 1) {
+    plan_kernel<<<1, PLAN_THREADS, smem, stream>>>(ids, w, R, E, seg, nullptr, 1, counts, offsets,
+                                                   perm, inv, w_sorted, status);
+    return cudaGetLastError();
+  }
+  plan_hist_kernel<<<grid, PLAN_THREADS, sizeof(int32_t) * E, stream>>>(ids, R, E, seg, scratch);
+  plan_kernel<<<grid, PLAN_THREADS, smem, stream>>>(ids, w, R, E, seg, scratch, grid, counts,
+                                                    offsets, perm, inv, w_sorted, status);
   return cudaGetLastError();
 }
 

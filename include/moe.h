@@ -93,7 +93,8 @@ typedef enum moe_op {
 int moe_abi_version(void);
 
 /* Bytes of device workspace `op` needs for this shape (always >= 256; the first
- * 256 bytes hold the device status word).  The workspace must be 256-byte
+ * 256 bytes hold the device status word; the plan also keeps per-chunk expert
+ * histograms there, 256 * (E + 1) int32).  The workspace must be 256-byte
  * aligned.  Its contents need no initialisation except that the status word
  * should read 0 before the first call (zero the buffer once, or call
  * moe_get_device_status once, which clears it). */
@@ -173,8 +174,12 @@ moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
  * the SwiGLU activations in bf16, the gate-weighted expert outputs in fp32)
  * live in the workspace (moe_workspace_size(MOE_OP_FFN_FUSED, ...)).
  *   n_c: thread blocks given to the memory stages (dispatch / combine) while the
- *   GEMM blocks run, [COMET] 4.2.2.  0 runs the stages as consecutive kernels;
+ *   GEMM blocks run, [COMET] 4.2.1-4.2.2.  0 runs the stages as consecutive
+ *   kernels; n_c >= 1 runs plan, then ONE persistent cooperative kernel with one
+ *   CTA per SM, of which n_c dispatch and combine while the rest run the GEMM
+ *   tiles, handing off through per-m-tile and per-token ready flags;
  *   -1 takes the value from the library's profiled table for this shape.
+ *   n_c must be below 65 and below the SM count.
  * H and F must be multiples of 64.
  */
 moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
@@ -205,7 +210,8 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
  *   status  int32 [1] device pointer (may be NULL): receives this call's device
  *           status word (a moe_status; MOE_ERR_BAD_EXPERT_ID etc.).
  * Limit: the intermediates of R = M*topk rows need
- *   256 + R*H*2 + R*F*2 + R*H*4 + R*4 bytes (each part rounded up to 256);
+ *   256 + 256*(E+1)*4 + R*H*2 + R*F*2 + R*H*4 + R*4 bytes (each part rounded
+ *   up to 256);
  * a shape that needs more than MOE_NOALLOC_SCRATCH_BYTES is rejected with
  * MOE_ERR_WORKSPACE_TOO_SMALL before anything is launched (e.g. H=7168, F=4096,
  * topk=8 fits up to M=163 tokens; H=4096, F=14336, topk=2 up to M=630).
@@ -226,8 +232,19 @@ moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const void* W2,
  * and clears it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error. */
 moe_status moe_get_device_status(void* ws, void* stream);
 
-/* Time limit, in nanoseconds, of every bounded device-side wait (default 2 s). */
+/* Time limit, in nanoseconds, of every bounded device-side wait (default 2 s).
+ * In the single-kernel layer (moe_ffn_fused with n_c > 0) the limit counts time
+ * without progress anywhere in the kernel, not the total wait. */
 void moe_set_wait_timeout_ns(uint64_t ns);
+
+/* Test hook for failure detection (no GPU fault is ever injected):
+ *   kind 0           off (default)
+ *   kind 1, index m  the single-kernel layer never publishes m-tile m as
+ *                    dispatched, so the GEMM tiles waiting for it run into the
+ *                    wait limit and the call ends with MOE_ERR_TIMEOUT in the
+ *                    device status, leaving the context usable.
+ * Process-wide; returns MOE_ERR_INVALID_ARG for an unknown kind. */
+moe_status moe_set_fault_injection(int32_t kind, int32_t index);
 
 /* Message of the last host-side error on this thread ("" if none). */
 const char* moe_last_error(void);

@@ -41,12 +41,15 @@ def test_abi_version(lib):
 
 
 def test_workspace_sizes(lib):
-    for op in (B.OP_PLAN, B.OP_DISPATCH, B.OP_GROUPED_GEMM, B.OP_COMBINE):
+    for op in (B.OP_DISPATCH, B.OP_GROUPED_GEMM, B.OP_COMBINE):
         assert B.moe_workspace_size(op, 4096, 4096, 14336, 8, 2) == 256
+    # the plan keeps up to 256 per-chunk histograms of E + 1 counters
+    assert B.moe_workspace_size(B.OP_PLAN, 4096, 0, 0, 8, 2) == 256 + 256 * 9 * 4
+    assert B.moe_workspace_size(B.OP_PLAN, 4096, 0, 0, 1024, 2) == 256 + 256 * 1025 * 4
     R, H, F = 8192, 4096, 14336
     fused = B.moe_workspace_size(B.OP_FFN_FUSED, 4096, H, F, 8, 2)
     assert fused >= 256 + R * H * 2 + R * F * 2 + R * H * 4 + R * 4
-    assert B.moe_workspace_size(B.OP_FFN_FUSED, 0, H, F, 8, 2) == 256
+    assert B.moe_workspace_size(B.OP_FFN_FUSED, 0, H, F, 8, 2) >= 256 + 256 * 9 * 4
 
 
 FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
@@ -118,6 +121,8 @@ def test_fused_validation(lib):
     assert f(*args(F=96)) == 2
     assert f(*args(topk=5)) == 1
     assert f(*args(n_c=-2)) == 1
+    assert lib.moe_set_fault_injection(7, 0) == 1
+    assert lib.moe_set_fault_injection(0, 0) == 0
     assert f(*args(ws=need - 1)) == 4
 
 
