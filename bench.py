@@ -50,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--n-c-sweep", default=None, dest="n_c_sweep",
+                    help="comma-separated n_c values: print one timing line per value "
+                         "(profiling for the n_c table) instead of the benchmark line")
     return ap.parse_args(argv)
 
 
@@ -254,6 +257,29 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+
+    if args.n_c_sweep:
+        for nc in [int(v) for v in args.n_c_sweep.split(",")]:
+            for _ in range(args.warmup):
+                flush.fill_(1)
+                B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=nc)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(1)
+                evs[i][0].record(stream)
+                B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=nc)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            st = B.moe_get_device_status(ws)
+            ms = [a.elapsed_time(b) for a, b in evs]
+            if rank == 0:
+                print(json.dumps({"workload": wl.name, "n_c": nc, "status": st,
+                                  "ms_per_step": statistics.mean(ms), "ms_min": min(ms),
+                                  "tokens_per_s": M / (statistics.mean(ms) / 1e3)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     for _ in range(args.warmup):
         flush.fill_(1)

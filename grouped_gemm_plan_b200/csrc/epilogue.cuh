@@ -1,0 +1,123 @@
+// epilogue.cuh -- coalesced row stores for the GEMM epilogues.
+//
+// After tcgen05.ld every epilogue thread holds a piece of ONE output row (TMEM
+// lane = row), so storing straight from registers makes each warp store touch 32
+// different rows with 16 bytes each: 32 partial-line transactions per
+// instruction.  Instead each warp passes its 32 row segments of 128 bytes
+// through a 4 KB shared-memory buffer and writes them back four rows per
+// instruction: eight lanes cover one row's 128 contiguous bytes, so every store
+// instruction writes four full 128-byte lines.
+//
+// The buffer is XOR-swizzled in 16-byte units (slot j of row r lives at
+// r * 8 + (j ^ (r & 7))), so both the row-wise writes and the column-wise reads
+// are free of bank conflicts.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Bytes of staging buffer per epilogue warp.
+constexpr int EPI_STAGE_BYTES_PER_WARP = 32 * 128;
+
+// `seg` is this thread's 128-byte row segment; `dst` where it goes (nullptr: the
+// row is not written).  `buf` is this warp's staging buffer (256 x 16 B).
+__device__ __forceinline__ void warp_store_rows128(const uint4 (&seg)[8], uint8_t* dst, uint4* buf,
+                                                   int lane) {
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) buf[lane * 8 + (j ^ (lane & 7))] = seg[j];
+  __syncwarp();
+  const unsigned long long mine = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int row = it * 4 + (lane >> 3);
+    const int c16 = lane & 7;
+    const unsigned long long d = __shfl_sync(0xffffffffu, mine, row);
+    const uint4 v = buf[row * 8 + (c16 ^ (row & 7))];
+    if (d != 0ull) reinterpret_cast<uint4*>(d)[c16] = v;
+  }
+}
+
+__device__ __forceinline__ void pack8_bf16(const float* v, float scale, uint4& out) {
+  out.x = pack_bf16x2(v[0] * scale, v[1] * scale);
+  out.y = pack_bf16x2(v[2] * scale, v[3] * scale);
+  out.z = pack_bf16x2(v[4] * scale, v[5] * scale);
+  out.w = pack_bf16x2(v[6] * scale, v[7] * scale);
+}
+
+__device__ __forceinline__ float silu_fast(float g) { return g / (1.0f + __expf(-g)); }
+
+// SwiGLU of 8 gate/up pairs -> 8 bf16.
+__device__ __forceinline__ void pack8_swiglu(const float* g, const float* u, uint4& out) {
+  out.x = pack_bf16x2(silu_fast(g[0]) * u[0], silu_fast(g[1]) * u[1]);
+  out.y = pack_bf16x2(silu_fast(g[2]) * u[2], silu_fast(g[3]) * u[3]);
+  out.z = pack_bf16x2(silu_fast(g[4]) * u[4], silu_fast(g[5]) * u[5]);
+  out.w = pack_bf16x2(silu_fast(g[6]) * u[6], silu_fast(g[7]) * u[7]);
+}
+
+// The epilogue of one 128-row accumulator tile (this warp: 32 of the rows).
+//   EPI = MOE_EPI_STORE           bf16 C[row, col0 + 0..255]     (4 segments)
+//         MOE_EPI_SWIGLU          bf16 C[row, col0 + 0..127] from gate cols
+//                                 0..127 and up cols 128..255    (2 segments)
+//         MOE_EPI_WEIGHT_SCATTER  fp32 C[dest, col0 + 0..255] * scale (8 segments)
+// t_row: TMEM address of this warp's lanes, accumulator column 0.
+// row_dst: byte address of this thread's output row at column col0 (nullptr: the
+// row is not written); n_left: output columns from col0 to the end of the row
+// (segments past it are skipped, n_left is a multiple of 64).
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, uint8_t* row_dst, int32_t n_left,
+                                              float scale, uint4* buf, int lane) {
+  if (EPI == MOE_EPI_SWIGLU) {
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {  // 64 output columns = 128 bytes per segment
+      float g[32], u[32];
+      uint4 seg[8];
+      tmem_ld32(t_row + c * 64, g);
+      tmem_ld32(t_row + 128 + c * 64, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_swiglu(g + 8 * q, u + 8 * q, seg[q]);
+      tmem_ld32(t_row + c * 64 + 32, g);
+      tmem_ld32(t_row + 128 + c * 64 + 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_swiglu(g + 8 * q, u + 8 * q, seg[4 + q]);
+      uint8_t* d = (row_dst != nullptr && c * 64 < n_left) ? row_dst + c * 128 : nullptr;
+      warp_store_rows128(seg, d, buf, lane);
+    }
+  } else if (EPI == MOE_EPI_STORE) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {  // 64 bf16 columns per segment
+      float v[32];
+      uint4 seg[8];
+      tmem_ld32(t_row + c * 64, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_bf16(v + 8 * q, 1.0f, seg[q]);
+      tmem_ld32(t_row + c * 64 + 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_bf16(v + 8 * q, 1.0f, seg[4 + q]);
+      uint8_t* d = (row_dst != nullptr && c * 64 < n_left) ? row_dst + c * 128 : nullptr;
+      warp_store_rows128(seg, d, buf, lane);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {  // 32 fp32 columns per segment
+      float v[32];
+      uint4 seg[8];
+      tmem_ld32(t_row + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        seg[q] = make_uint4(__float_as_uint(v[4 * q] * scale), __float_as_uint(v[4 * q + 1] * scale),
+                            __float_as_uint(v[4 * q + 2] * scale),
+                            __float_as_uint(v[4 * q + 3] * scale));
+      uint8_t* d = (row_dst != nullptr && c * 32 < n_left) ? row_dst + c * 128 : nullptr;
+      warp_store_rows128(seg, d, buf, lane);
+    }
+  }
+}
+
+}  // namespace moe

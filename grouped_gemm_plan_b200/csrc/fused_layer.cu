@@ -24,6 +24,7 @@
 // flag and lets every CTA leave cleanly (in-flight TMA loads landed, MMAs
 // drained, TMEM freed).
 #include "common.cuh"
+#include "epilogue.cuh"
 
 namespace moe {
 
@@ -39,7 +40,7 @@ constexpr int L_A_BYTES = L_BM * L_BK * 2;
 constexpr int L_B_BOX_BYTES = L_BK * 64 * 2;
 constexpr int L_STAGE_BYTES = L_A_BYTES + 4 * L_B_BOX_BYTES;
 constexpr int L_TMEM_COLS = 512;
-constexpr int L_DYN_SMEM = L_STAGES * L_STAGE_BYTES + 1024;
+constexpr int L_DYN_SMEM = L_STAGES * L_STAGE_BYTES + 4 * EPI_STAGE_BYTES_PER_WARP + 1024;
 constexpr uint32_t L_IDESC = idesc_bf16_f32(L_BM, L_BN, true);
 
 }  // namespace
@@ -155,8 +156,6 @@ __device__ __forceinline__ void give_up(const LayerArgs& a, volatile int32_t* sa
   atomicExch(a.sync.abort, 1);
   *sabort = 1;
 }
-
-__device__ __forceinline__ float silu_l(float g) { return g / (1.0f + __expf(-g)); }
 
 __global__ void __launch_bounds__(L_THREADS, 1)
     moe_layer_kernel(const __grid_constant__ CUtensorMap tmXp,
@@ -433,6 +432,8 @@ __global__ void __launch_bounds__(L_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    uint4* stage_buf = reinterpret_cast<uint4*>(ring + L_STAGES * L_STAGE_BYTES +
+                                                (warp - 2) * EPI_STAGE_BYTES_PER_WARP);
     uint32_t j = 0;
     for (int32_t t = g; t < T; t += G, ++j) {
       const bool two = t >= T1;
@@ -452,27 +453,10 @@ __global__ void __launch_bounds__(L_THREADS, 1)
       const bool row_ok = r < tc.rows;
       const int32_t s = tc.row0 + r;
       if (!two) {
-        __nv_bfloat16* dst = a.h + static_cast<int64_t>(s) * a.F;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float gv[32], uv[32];
-          tmem_ld32(t_row + c * 32, gv);
-          tmem_ld32(t_row + 128 + c * 32, uv);
-          tmem_ld_wait();
-          const int32_t col = tc.ni * 128 + c * 32;
-          if (row_ok && col < a.F) {
-            uint4* d = reinterpret_cast<uint4*>(dst + col);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              uint4 u;
-              u.x = pack_bf16x2(silu_l(gv[8 * qq + 0]) * uv[8 * qq + 0], silu_l(gv[8 * qq + 1]) * uv[8 * qq + 1]);
-              u.y = pack_bf16x2(silu_l(gv[8 * qq + 2]) * uv[8 * qq + 2], silu_l(gv[8 * qq + 3]) * uv[8 * qq + 3]);
-              u.z = pack_bf16x2(silu_l(gv[8 * qq + 4]) * uv[8 * qq + 4], silu_l(gv[8 * qq + 5]) * uv[8 * qq + 5]);
-              u.w = pack_bf16x2(silu_l(gv[8 * qq + 6]) * uv[8 * qq + 6], silu_l(gv[8 * qq + 7]) * uv[8 * qq + 7]);
-              d[qq] = u;
-            }
-          }
-        }
+        const int32_t col0 = tc.ni * 128;
+        uint8_t* dst = row_ok ? reinterpret_cast<uint8_t*>(a.h + static_cast<int64_t>(s) * a.F + col0)
+                              : nullptr;
+        epilogue_tile<MOE_EPI_SWIGLU>(t_row, dst, a.F - col0, 1.0f, stage_buf, lane);
         tc_fence_before();
         mbar_arrive(&tempty_bar[b]);
         // publish this warp's 32 rows of the m-tile's column block
@@ -484,6 +468,7 @@ __global__ void __launch_bounds__(L_THREADS, 1)
           if (q == 2) red_release_add(sy.progress, 1);
         }
       } else {
+        const int32_t col0 = tc.ni * L_BN;
         float scale = 1.0f;
         int32_t dest = -1;
         if (row_ok) {
@@ -494,23 +479,14 @@ __global__ void __launch_bounds__(L_THREADS, 1)
             dest = -1;
           }
         }
-        float* dst = a.yk + static_cast<int64_t>(dest < 0 ? 0 : dest) * a.H;
-#pragma unroll 1
-        for (int c = 0; c < L_BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(t_row + c * 32, v);
-          tmem_ld_wait();
-          const int32_t col = tc.ni * L_BN + c * 32;
-          if (dest >= 0 && col < a.H) {
-            float4* d = reinterpret_cast<float4*>(dst + col);
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq)
-              d[qq] = make_float4(v[4 * qq] * scale, v[4 * qq + 1] * scale, v[4 * qq + 2] * scale,
-                                  v[4 * qq + 3] * scale);
-          }
-        }
+        uint8_t* dst = dest >= 0 ? reinterpret_cast<uint8_t*>(a.yk + static_cast<int64_t>(dest) * a.H + col0)
+                                 : nullptr;
+        epilogue_tile<MOE_EPI_WEIGHT_SCATTER>(t_row, dst, a.H - col0, scale, stage_buf, lane);
         tc_fence_before();
         mbar_arrive(&tempty_bar[b]);
+        // The warp wrote its rows' segments cooperatively: order them before the
+        // per-row completion counts of the lanes that own the rows.
+        __syncwarp();
         if (dest >= 0) {
           // row complete once all nt2 column tiles wrote it; token complete once
           // all its topk rows are complete

@@ -14,6 +14,14 @@ from helpers import check_stage, guarded_empty
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True, params=["single", "pair"])
+def gemm_kernel(request, monkeypatch):
+    """Run every test on both grouped GEMM kernels: single-CTA 128-row tiles and
+    CTA-pair (tcgen05 cta_group::2) 256-row tiles."""
+    monkeypatch.setenv("MOE_GEMM_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
+
+
 def _offsets(counts):
     return np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
 

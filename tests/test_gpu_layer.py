@@ -123,6 +123,14 @@ def test_layer_bad_expert_id(cuda_dev):
     assert counts.cpu().tolist() == [0] * 4
 
 
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_layer_both_gemm_kernels(cuda_dev, monkeypatch, pair):
+    monkeypatch.setenv("MOE_GEMM_PAIR", pair)
+    w, x, W1, W2, ids, tw = layer_case(700, 512, 384, 4, 2, "skewed", seed=12)
+    out = run_fused(cuda_dev, x, W1, W2, ids, tw)[0]
+    check_close(out, oracle.moe_ffn(x, W1, W2, ids, tw), f"layer, pair kernel={pair}")
+
+
 def test_layer_deterministic(cuda_dev):
     w, x, W1, W2, ids, tw = layer_case(777, 512, 384, 16, 2, "skewed", seed=5)
     a = run_fused(cuda_dev, x, W1, W2, ids, tw)[0]

@@ -18,6 +18,13 @@ from test_gpu_layer import run_fused
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(autouse=True)
+def single_cta_sequence(monkeypatch):
+    """The single-kernel layer uses 128-row tiles; the five-launch reference it is
+    compared with bit for bit is pinned to the single-CTA GEMM (same tiles)."""
+    monkeypatch.setenv("MOE_GEMM_PAIR", "0")
+
 CASES = [
     (256, 256, 512, 8, 2, "uniform"),
     (129, 512, 192, 3, 3, "skewed"),
