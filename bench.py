@@ -16,7 +16,6 @@ barrier and the max-over-ranks of the timings.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import os
@@ -68,64 +67,103 @@ def peaks():
 # ---------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
-              "clocks_event_reasons.sw_power_cap"]
+    """SM clock and throttle reasons sampled while the timed region runs.
 
-    def __init__(self, index: int):
+    Reads NVML from a background thread every 5 ms (read-only queries; nothing is
+    set), so a timed region of tens of milliseconds still gets a dozen samples.
+    Falls back to `nvidia-smi -lms 200` when NVML is not importable.
+    """
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
         self.index = index
-        self.proc = None
-        self.lines: list[str] = []
-        self.thread = None
+        self.period = period_s
+        self.samples: list[tuple[float, int, float]] = []  # (mhz, reason bits, watts)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        self._proc = None
+        self._lines: list[str] = []
 
     def start(self):
         try:
-            cmd = ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._poll_nvml, args=(h,), daemon=True)
+            self._thread.start()
+            return
+        except Exception:
+            self._nvml = None
+        try:
+            cmd = ["nvidia-smi", f"--id={self.index}", "--query-gpu=clocks.sm,clocks.max.sm",
                    "--format=csv,noheader,nounits", "-lms", "200"]
             if shutil.which("stdbuf"):
-                cmd = ["stdbuf", "-oL"] + cmd      # one line per sample, not one block at exit
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True, bufsize=1)
+                cmd = ["stdbuf", "-oL"] + cmd
+            self._proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                          text=True, bufsize=1)
+            self._thread = threading.Thread(target=self._read_smi, daemon=True)
+            self._thread.start()
         except OSError:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
-        self.thread.start()
+            self._proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll_nvml(self, h):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((float(mhz), int(bits), watts))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def _read_smi(self):
+        for line in self._proc.stdout:
+            self._lines.append(line.strip())
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.3)                      # one more sample period
-        self.proc.send_signal(signal.SIGINT)
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            self.proc.wait(timeout=5)
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        self._stop.set()
+        if self._proc is not None:
+            time.sleep(0.3)
+            self._proc.send_signal(signal.SIGINT)
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        reasons = set()
+        if self._nvml is not None:
+            for name, const in self.REASONS.items():
+                bit = getattr(self._nvml, const, 0)
+                if any(b & bit for _, b, _ in self.samples):
+                    reasons.add(name)
+            mhz = [m for m, _, _ in self.samples]
+            watts = [w for _, _, w in self.samples]
+            return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                    "sm_mhz_min": min(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                    "power_w_max": max(watts) if watts else None,
+                    "reasons": sorted(reasons), "samples": len(mhz), "source": "nvml 5 ms"}
+        sm, smax = [], []
+        for line in self._lines:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
             try:
                 sm.append(float(parts[0]))
                 smax.append(float(parts[1]))
-            except ValueError:
+            except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, parts[3:]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_max_mhz": max(smax) if smax else None, "reasons": [],
+                "samples": len(sm), "source": "nvidia-smi 200 ms (reasons not sampled)"}
 
 
 # ---------------------------------------------------------------------------- oracle arm
@@ -214,23 +252,19 @@ def measured_traffic(kernel: str, workload: str):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     from grouped_gemm_plan_b200 import binding as B
+    from grouped_gemm_plan_b200 import dist as D
     from grouped_gemm_plan_b200 import workload as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = D.env_rank()
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    D.init("nccl", timeout_s=120, device=dev)
     B.load()
 
-    wl = W.rank_workload(W.WORKLOADS[args.workload], rank)
+    wl = D.shard(W.WORKLOADS[args.workload], rank)
     M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
     x_h = W.make_x(wl).pin_memory()
     ids_np, tw_np = W.make_routing(wl)
@@ -254,9 +288,7 @@ def run_ours(args):
         B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=args.n_c)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
+        D.barrier(dev)
 
     if args.n_c_sweep:
         for nc in [int(v) for v in args.n_c_sweep.split(",")]:
@@ -277,8 +309,7 @@ def run_ours(args):
                 print(json.dumps({"workload": wl.name, "n_c": nc, "status": st,
                                   "ms_per_step": statistics.mean(ms), "ms_min": min(ms),
                                   "tokens_per_s": M / (statistics.mean(ms) / 1e3)}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
+        D.finish()
         return 0
 
     for _ in range(args.warmup):
@@ -358,13 +389,10 @@ def run_ours(args):
     d2h = out_h.numel() * 2
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = D.max_over_ranks([total_ms, e2e_ms], dev)
     ms_per_step = total_ms / args.steps
-    value = world * M * args.steps / (total_ms / 1e3)
-    e2e_value = world * M * args.steps / (e2e_ms / 1e3)
+    value = D.whole_job_rate(M * args.steps, world, total_ms / 1e3)
+    e2e_value = D.whole_job_rate(M * args.steps, world, e2e_ms / 1e3)
 
     pk, pk_kind = peaks()
     flops_g1 = 4.0 * R * H * F
@@ -421,9 +449,7 @@ def run_ours(args):
             **extra,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    D.finish()
     return 0
 
 
