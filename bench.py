@@ -82,7 +82,8 @@ class ClockSampler:
     def __init__(self, index: int, period_s: float = 0.005):
         self.index = index
         self.period = period_s
-        self.samples: list[tuple[float, int, float]] = []  # (mhz, reason bits, watts)
+        self.samples: list[tuple[float, float, int, float]] = []  # (t, mhz, reason bits, watts)
+        self.window = (0.0, float("inf"))
         self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
@@ -90,7 +91,12 @@ class ClockSampler:
         self._proc = None
         self._lines: list[str] = []
 
+    def mark(self, t0: float, t1: float):
+        """Keep only samples taken between host times t0 and t1 (time.monotonic())."""
+        self.window = (t0, t1)
+
     def start(self):
+        sys.setswitchinterval(0.0005)   # let the polling thread run between launches
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -118,10 +124,11 @@ class ClockSampler:
         nv = self._nvml
         while not self._stop.is_set():
             try:
+                t = time.monotonic()
                 mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((float(mhz), int(bits), watts))
+                self.samples.append((t, float(mhz), int(bits), watts))
             except Exception:
                 pass
             self._stop.wait(self.period)
@@ -141,14 +148,17 @@ class ClockSampler:
                 self._proc.kill()
         if self._thread is not None:
             self._thread.join(timeout=5)
+        sys.setswitchinterval(0.005)
         reasons = set()
         if self._nvml is not None:
+            t0, t1 = self.window
+            inside = [x for x in self.samples if t0 <= x[0] <= t1]
             for name, const in self.REASONS.items():
                 bit = getattr(self._nvml, const, 0)
-                if any(b & bit for _, b, _ in self.samples):
+                if any(b & bit for _, _, b, _ in inside):
                     reasons.add(name)
-            mhz = [m for m, _, _ in self.samples]
-            watts = [w for _, _, w in self.samples]
+            mhz = [m for _, m, _, _ in inside]
+            watts = [w for _, _, _, w in inside]
             return {"sm_mhz": statistics.median(mhz) if mhz else None,
                     "sm_mhz_min": min(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
                     "power_w_max": max(watts) if watts else None,
@@ -231,9 +241,17 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------- our arm
 
-def source_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+GEMM_SOURCES = ["grouped_gemm.cu", "epilogue.cuh", "common.cuh"]
+
+
+def kernel_sources_sha() -> str:
+    """Hash of the sources the measured GEMM kernel is built from: a recorded DRAM
+    traffic figure is used only while these are unchanged."""
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "grouped_gemm_plan_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(kernel: str, workload: str):
@@ -242,8 +260,7 @@ def measured_traffic(kernel: str, workload: str):
             rows = json.load(f)
     except (OSError, ValueError):
         return None
-    src = os.path.join(ROOT, "grouped_gemm_plan_b200", "csrc", "grouped_gemm.cu")
-    sha = source_sha(src)
+    sha = kernel_sources_sha()
     for r in rows:
         if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_sha") == sha:
             return r.get("dram_bytes_per_launch")
@@ -312,6 +329,8 @@ def run_ours(args):
         D.finish()
         return 0
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         flush.fill_(1)
         step()
@@ -320,17 +339,17 @@ def run_ours(args):
         raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} after warm-up")
 
     # ---- timed region: K steps, L2 flushed before each, device time by CUDA events
-    clocks = ClockSampler(local)
-    clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
+    t_begin = time.monotonic()
     for i in range(args.steps):
         flush.fill_(1)
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     barrier()
+    clocks.mark(t_begin, time.monotonic())
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
