@@ -20,28 +20,40 @@ namespace moe {
 
 constexpr int PM_THREADS = 256;
 
-// Work item = (row s, step q): lane l of the warp copies 16-byte vector
-// q*32 + l of the row.  Splitting rows into 512-byte steps keeps every SM busy
-// even when there are only a few rows (small batches).
+// Work item = (row s, step group q): lane l of the warp copies 16-byte vectors
+// (q*DU + u)*32 + l of the row, u < DU, all DU loads issued before the stores.
+// Splitting rows into 2 KB groups keeps every SM busy even when there are only a
+// few rows (small batches) and keeps DU loads in flight per lane.
+constexpr int DU = 4;
+
 __global__ void __launch_bounds__(PM_THREADS)
     dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int32_t R,
                     int32_t topk, int32_t vpr, uint4* __restrict__ xp, int32_t* status) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
-  const int32_t steps = (vpr + 31) >> 5;
-  const int64_t items = static_cast<int64_t>(R) * steps;
+  const int32_t groups = (vpr + 32 * DU - 1) / (32 * DU);
+  const int64_t items = static_cast<int64_t>(R) * groups;
   for (int64_t it = (static_cast<int64_t>(blockIdx.x) * PM_THREADS + threadIdx.x) >> 5; it < items;
        it += nwarps) {
-    const int32_t s = static_cast<int32_t>(it / steps);
-    const int32_t c = static_cast<int32_t>(it - static_cast<int64_t>(s) * steps) * 32 + lane;
+    const int32_t s = static_cast<int32_t>(it / groups);
+    const int32_t c0 = static_cast<int32_t>(it - static_cast<int64_t>(s) * groups) * (32 * DU) + lane;
     const int32_t i = __ldg(perm + s);
     uint4* dst = xp + static_cast<int64_t>(s) * vpr;
     if (i < 0 || i >= R) {
       if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
-      if (c < vpr) dst[c] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < DU; ++u)
+        if (c0 + 32 * u < vpr) dst[c0 + 32 * u] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    if (c < vpr) dst[c] = __ldg(x + static_cast<int64_t>(i / topk) * vpr + c);
+    const uint4* src = x + static_cast<int64_t>(i / topk) * vpr;
+    uint4 v[DU];
+#pragma unroll
+    for (int u = 0; u < DU; ++u)
+      if (c0 + 32 * u < vpr) v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+    for (int u = 0; u < DU; ++u)
+      if (c0 + 32 * u < vpr) dst[c0 + 32 * u] = v[u];
   }
 }
 
@@ -102,13 +114,15 @@ __global__ void __launch_bounds__(PM_THREADS)
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
   const int64_t row_bytes = static_cast<int64_t>(vpr) * (F32 ? 32 : 16);
-  const int32_t steps = (vpr + 31) >> 5;
-  const int64_t items = static_cast<int64_t>(M) * steps;
-  // Work item = (token t, step q): lane l handles group q*32 + l of eight elements.
+  constexpr int CU = KMAX <= 8 ? 2 : 1;  // steps per work item: CU * topk loads in flight
+  const int32_t groups = (vpr + 32 * CU - 1) / (32 * CU);
+  const int64_t items = static_cast<int64_t>(M) * groups;
+  // Work item = (token t, step group q): lane l handles groups of eight elements
+  // (q*CU + u)*32 + l, u < CU.
   for (int64_t it = (static_cast<int64_t>(blockIdx.x) * PM_THREADS + threadIdx.x) >> 5; it < items;
        it += nwarps) {
-    const int32_t t = static_cast<int32_t>(it / steps);
-    const int32_t c = static_cast<int32_t>(it - static_cast<int64_t>(t) * steps) * 32 + lane;
+    const int32_t t = static_cast<int32_t>(it / groups);
+    const int32_t cbase = static_cast<int32_t>(it - static_cast<int64_t>(t) * groups) * (32 * CU) + lane;
     int32_t my_row = 0;
     float my_w = 1.0f;
     if (lane < topk) {
@@ -127,25 +141,44 @@ __global__ void __launch_bounds__(PM_THREADS)
       rows[k] = __shfl_sync(0xffffffffu, my_row, k);
       wk[k] = __shfl_sync(0xffffffffu, my_w, k);
     }
-    if (c >= vpr) continue;
-    Vec8<F32> v[KMAX];
+    constexpr int KC = KMAX < 8 ? KMAX : 8;  // top-k rows loaded per batch
+    float acc[CU][8];
 #pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-      if (k < topk && rows[k] >= 0)
-        v[k].load(y + static_cast<int64_t>(rows[k]) * row_bytes, c);
-      else
-        v[k].zero();
+    for (int u = 0; u < CU; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < KMAX; k0 += KC) {
+      Vec8<F32> v[CU][KC];
+#pragma unroll
+      for (int u = 0; u < CU; ++u) {
+        const int32_t c = cbase + 32 * u;
+#pragma unroll
+        for (int kk = 0; kk < KC; ++kk) {
+          const int k = k0 + kk;
+          if (c < vpr && k < topk && rows[k] >= 0)
+            v[u][kk].load(y + static_cast<int64_t>(rows[k]) * row_bytes, c);
+          else
+            v[u][kk].zero();
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < CU; ++u)
+#pragma unroll
+        for (int kk = 0; kk < KC; ++kk)
+          if (k0 + kk < topk) v[u][kk].fma_into(acc[u], wk[k0 + kk]);
     }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < KMAX; ++k)
-      if (k < topk) v[k].fma_into(acc, wk[k]);
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    out[static_cast<int64_t>(t) * vpr + c] = o;
+    for (int u = 0; u < CU; ++u) {
+      const int32_t c = cbase + 32 * u;
+      if (c >= vpr) continue;
+      uint4 o;
+      o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+      o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+      o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+      o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      out[static_cast<int64_t>(t) * vpr + c] = o;
+    }
   }
 }
 
@@ -161,8 +194,8 @@ cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream) {
   const int64_t R = M * topk;
   if (R == 0) return cudaSuccess;
-  const int64_t steps = (H / 8 + 31) / 32;
-  dispatch_kernel<<<grid_for_items(R * steps, num_sms), PM_THREADS, 0, stream>>>(
+  const int64_t groups = (H / 8 + 32 * DU - 1) / (32 * DU);
+  dispatch_kernel<<<grid_for_items(R * groups, num_sms), PM_THREADS, 0, stream>>>(
       reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
       static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
   return cudaGetLastError();
