@@ -300,6 +300,9 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     return fail(MOE_ERR_MISALIGNED, "x, W1, W2 and out must be 16-byte aligned");
 
   const int64_t R = M * topk;
+  // Overlapping kernel boundaries pays off on small layers only (measured).
+  moe::PdlScope pdl(static_cast<double>(R) * static_cast<double>(H) * static_cast<double>(F) <
+                    4294967296.0);
   const FusedLayout L = fused_layout(M, H, F, E, topk);
   uint8_t* base = static_cast<uint8_t*>(ws);
   void* xp = base + L.xp;

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstdlib>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -94,6 +95,67 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+//
+// Kernels can be launched with programmatic stream serialisation: a kernel may
+// then start while the previous kernel on the stream is finishing, runs only its
+// prologue (shared-memory barriers, TMEM, tensor-map prefetch), and waits in
+// griddep_wait() -- until the previous grid has completed and its memory is
+// visible -- before its first global read or write.  Launched without it, the
+// wait returns at once.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel on the stream be scheduled once every CTA of this grid has
+// issued it or exited (the next kernel still waits in griddep_wait for this grid
+// to finish).  The short kernels issue it at their start; the GEMM kernels when a
+// CTA starts its last tile, so that waiting CTAs of the next kernel do not sit on
+// the SMs for the whole GEMM.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Whether the launches of the current call use programmatic serialisation.  The
+// layer call turns it on for small layers, where kernel boundaries are a visible
+// share of the step; measured on large layers it slowed the GEMMs down, so there
+// (and in the single-stage calls) kernels are launched in plain stream order.
+inline thread_local bool g_pdl_enabled = false;
+
+struct PdlScope {
+  bool saved;
+  explicit PdlScope(bool on) : saved(g_pdl_enabled) {
+    const char* v = getenv("MOE_PDL");  // MOE_PDL=0/1 forces it off/on (comparisons)
+    g_pdl_enabled = (v != nullptr && (v[0] == '0' || v[0] == '1')) ? (v[0] == '1') : on;
+  }
+  ~PdlScope() { g_pdl_enabled = saved; }
+};
+
+// cudaLaunchKernelEx with programmatic stream serialisation when enabled (plus an
+// optional cluster shape).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = g_pdl_enabled ? 1 : 0;
+  unsigned n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
 // ---------------------------------------------------------------- cross-CTA flags

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     tmem_alloc(&s_tmem_base, G_TMEM_COLS);
     tmem_relinquish();
   }
+  griddep_wait();  // offsets and A are written by the kernels before this one
   for (int e = tid; e <= E; e += G_THREADS) s_off[e] = args.offsets[e];
   __syncthreads();
 
@@ -187,6 +188,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     uint32_t stage = 0, phase = 0;
     uint32_t issued = 0;
     for (int32_t t = blockIdx.x; t < T && !s_abort; t += gridDim.x) {
+      // the next kernel may be scheduled once every CTA is on its last tile
+      if (t + static_cast<int32_t>(gridDim.x) >= T) griddep_launch_dependents();
       const TileCoord tc = decode_tile(t, s_tstart, s_off, E, args.n_tiles_n);
       for (int32_t kb = 0; kb < KB; ++kb) {
         if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.timeout_ns, &s_abort)) {
@@ -469,21 +472,23 @@ static int launch_grouped_gemm_1sm(const void* A, const void* B, const int32_t* 
     case MOE_EPI_SWIGLU:
       err = set_gemm_attr_once<MOE_EPI_SWIGLU>();
       if (err != cudaSuccess) return 2;
-      grouped_gemm_kernel<MOE_EPI_SWIGLU><<<grid, G_THREADS, G_DYN_SMEM, stream>>>(tmA, tmB, a);
+      err = launch_pdl(grouped_gemm_kernel<MOE_EPI_SWIGLU>, dim3(grid), dim3(G_THREADS), G_DYN_SMEM,
+                       stream, 1, tmA, tmB, a);
       break;
     case MOE_EPI_WEIGHT_SCATTER:
       err = set_gemm_attr_once<MOE_EPI_WEIGHT_SCATTER>();
       if (err != cudaSuccess) return 2;
-      grouped_gemm_kernel<MOE_EPI_WEIGHT_SCATTER>
-          <<<grid, G_THREADS, G_DYN_SMEM, stream>>>(tmA, tmB, a);
+      err = launch_pdl(grouped_gemm_kernel<MOE_EPI_WEIGHT_SCATTER>, dim3(grid), dim3(G_THREADS),
+                       G_DYN_SMEM, stream, 1, tmA, tmB, a);
       break;
     default:
       err = set_gemm_attr_once<MOE_EPI_STORE>();
       if (err != cudaSuccess) return 2;
-      grouped_gemm_kernel<MOE_EPI_STORE><<<grid, G_THREADS, G_DYN_SMEM, stream>>>(tmA, tmB, a);
+      err = launch_pdl(grouped_gemm_kernel<MOE_EPI_STORE>, dim3(grid), dim3(G_THREADS), G_DYN_SMEM,
+                       stream, 1, tmA, tmB, a);
       break;
   }
-  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+  return err == cudaSuccess ? 0 : 2;
 }
 
 }  // namespace moe

@@ -223,6 +223,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     tmem_alloc2(&s_tmem_base, P_TMEM_COLS);
     tmem_relinquish2();
   }
+  griddep_wait();  // offsets and A are written by the kernels before this one
   for (int e = tid; e <= E; e += P_THREADS) s_off[e] = args.offsets[e];
   __syncthreads();
   if (warp == 0) {
@@ -263,6 +264,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     uint32_t stage = 0, phase = 0;
     bool issued_any = false;
     for (int32_t t = pair; t < T && !s_abort; t += npairs) {
+      // the next kernel may be scheduled once every CTA is on its last tile
+      if (t + npairs >= T) griddep_launch_dependents();
       const PTile tc = decode2(t, s_tstart, s_off, E);
       const int32_t arow = tc.row0 + 128 * static_cast<int32_t>(rank);
       for (int32_t kb = 0; kb < KB; ++kb) {
@@ -462,19 +465,8 @@ static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& 
     if (err != cudaSuccess) return err;
     if (dev < 31) mask |= (1 << dev);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(P_THREADS);
-  cfg.dynamicSmemBytes = P_DYN_SMEM;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_2sm_kernel<EPI>, a, b, args);
+  return launch_pdl(grouped_gemm_2sm_kernel<EPI>, dim3(static_cast<unsigned>(grid)), dim3(P_THREADS),
+                    P_DYN_SMEM, stream, 2, a, b, args);
 }
 
 // Same contract as launch_grouped_gemm (0 ok, 1 tensor map, 2 CUDA error).

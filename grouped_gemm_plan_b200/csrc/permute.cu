@@ -29,6 +29,8 @@ constexpr int DU = 4;
 __global__ void __launch_bounds__(PM_THREADS)
     dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int32_t R,
                     int32_t topk, int32_t vpr, uint4* __restrict__ xp, int32_t* status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
   const int32_t groups = (vpr + 32 * DU - 1) / (32 * DU);
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(PM_THREADS)
     combine_kernel(const uint8_t* __restrict__ y, const int32_t* __restrict__ inv,
                    const float* __restrict__ w, int32_t M, int32_t R, int32_t topk,
                    int32_t vpr, uint4* __restrict__ out, int32_t* status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
   const int64_t row_bytes = static_cast<int64_t>(vpr) * (F32 ? 32 : 16);
@@ -195,26 +199,27 @@ cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64
   const int64_t R = M * topk;
   if (R == 0) return cudaSuccess;
   const int64_t groups = (H / 8 + 32 * DU - 1) / (32 * DU);
-  dispatch_kernel<<<grid_for_items(R * groups, num_sms), PM_THREADS, 0, stream>>>(
-      reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
-      static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_kernel, dim3(grid_for_items(R * groups, num_sms)), dim3(PM_THREADS), 0,
+                    stream, 1, reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
+                    static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
 }
 
 template <bool F32>
-static void launch_combine_t(int grid, cudaStream_t stream, const uint8_t* y, const int32_t* inv,
+static cudaError_t launch_combine_t(int grid, cudaStream_t stream, const uint8_t* y, const int32_t* inv,
                              const float* w, int32_t m, int32_t R, int32_t topk, int32_t vpr,
                              uint4* ov, int32_t* status) {
+  cudaError_t err;
   if (topk <= 2)
-    combine_kernel<2, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+    err = launch_pdl(combine_kernel<2, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
   else if (topk <= 4)
-    combine_kernel<4, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+    err = launch_pdl(combine_kernel<4, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
   else if (topk <= 8)
-    combine_kernel<8, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+    err = launch_pdl(combine_kernel<8, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
   else if (topk <= 16)
-    combine_kernel<16, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+    err = launch_pdl(combine_kernel<16, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
   else
-    combine_kernel<32, F32><<<grid, PM_THREADS, 0, stream>>>(y, inv, w, m, R, topk, vpr, ov, status);
+    err = launch_pdl(combine_kernel<32, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
+  return err;
 }
 
 cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
@@ -227,11 +232,8 @@ cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const 
   const uint8_t* yb = reinterpret_cast<const uint8_t*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out);
   const int32_t m = static_cast<int32_t>(M);
-  if (y_f32)
-    launch_combine_t<true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
-  else
-    launch_combine_t<false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
-  return cudaGetLastError();
+  return y_f32 ? launch_combine_t<true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status)
+               : launch_combine_t<false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
 }
 
 }  // namespace moe

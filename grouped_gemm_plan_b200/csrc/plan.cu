@@ -42,8 +42,10 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   const int32_t chunk = PLAN_WARPS * seg;
   const int32_t c0 = blockIdx.x * chunk;
   const int32_t c1 = min(c0 + chunk, R);
+  griddep_launch_dependents();
   for (int e = tid; e < E; e += PLAN_THREADS) hist_smem[e] = 0;
   if (tid == 0) s_bad = 0;
+  griddep_wait();
   __syncthreads();
   for (int32_t base = c0; base < c1; base += PLAN_THREADS) {
     const int32_t i = base + tid;
@@ -77,12 +79,14 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   const int32_t c0 = blockIdx.x * chunk;
   const int32_t c1 = min(c0 + chunk, R);
 
+  griddep_launch_dependents();
   for (int e = tid; e < E; e += PLAN_THREADS) {
     tot[e] = 0;
     before[e] = 0;
   }
   for (int j = tid; j < PLAN_WARPS * E; j += PLAN_THREADS) wbase[j] = 0;
   if (tid == 0) s_bad = 0;
+  griddep_wait();
   __syncthreads();
 
   if (hist != nullptr) {
@@ -230,9 +234,9 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
   }
   if (R == 0) {
     // Only counts/offsets to write: one CTA with no rows.
-    plan_kernel<<<1, PLAN_THREADS, smem, stream>>>(ids, w, 0, E, 32, nullptr, 0, counts, offsets,
-                                                   perm, inv, w_sorted, status);
-    return cudaGetLastError();
+    return launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), smem, stream, 1, ids, w, 0, E, 32,
+                      static_cast<const int32_t*>(nullptr), 0, counts, offsets, perm, inv, w_sorted,
+                      status);
   }
   const int max_chunks = num_sms < PLAN_MAX_CHUNKS ? num_sms : PLAN_MAX_CHUNKS;
   int32_t per_cta = (R + max_chunks - 1) / max_chunks;
@@ -242,14 +246,16 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
   const int32_t chunk = seg * PLAN_WARPS;
   const int32_t grid = (R + chunk - 1) / chunk;
   if (grid == 1) {
-    plan_kernel<<<1, PLAN_THREADS, smem, stream>>>(ids, w, R, E, seg, nullptr, 1, counts, offsets,
-                                                   perm, inv, w_sorted, status);
-    return cudaGetLastError();
+    return launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), smem, stream, 1, ids, w, R, E, seg,
+                      static_cast<const int32_t*>(nullptr), 1, counts, offsets, perm, inv, w_sorted,
+                      status);
   }
-  plan_hist_kernel<<<grid, PLAN_THREADS, sizeof(int32_t) * E, stream>>>(ids, R, E, seg, scratch);
-  plan_kernel<<<grid, PLAN_THREADS, smem, stream>>>(ids, w, R, E, seg, scratch, grid, counts,
-                                                    offsets, perm, inv, w_sorted, status);
-  return cudaGetLastError();
+  cudaError_t err = launch_pdl(plan_hist_kernel, dim3(grid), dim3(PLAN_THREADS), sizeof(int32_t) * E,
+                               stream, 1, ids, R, E, seg, scratch);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(plan_kernel, dim3(grid), dim3(PLAN_THREADS), smem, stream, 1, ids, w, R, E, seg,
+                    static_cast<const int32_t*>(scratch), grid, counts, offsets, perm, inv, w_sorted,
+                    status);
 }
 
 }  // namespace moe
