@@ -408,6 +408,22 @@ def run_ours(args):
     assert torch.equal(out_chain.view(torch.int16), out.view(torch.int16)), \
         "stage-by-stage result differs from the layer call"
 
+    # ---- the router in front of the layer (moe_route): fp32 logits [M, E] -> ids, w
+    g = torch.Generator(device=dev).manual_seed(wl.seed)
+    logits = torch.randn((M, E), generator=g, device=dev, dtype=torch.float32)
+    r_ids = torch.empty((M, topk), dtype=torch.int32, device=dev)
+    r_w = torch.empty((M, topk), dtype=torch.float32, device=dev)
+    r_ws = B.alloc_workspace(B.OP_ROUTE, M, 0, 0, E, topk, dev)
+    rev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    B.moe_route(logits, topk, r_ids, r_w, r_ws)
+    rev[0].record(stream)
+    for _ in range(10):
+        B.moe_route(logits, topk, r_ids, r_w, r_ws)
+    rev[1].record(stream)
+    torch.cuda.synchronize()
+    router_us = rev[0].elapsed_time(rev[1]) * 100.0
+    assert B.moe_get_device_status(r_ws) == B.MOE_OK
+
     # ---- end to end: every step's inputs are copied in from pinned host memory and
     # its result copied back, through the public call.  As in a serving loop, step
     # i+1's upload (one copy stream) and step i-1's download (another) overlap step
@@ -500,6 +516,7 @@ def run_ours(args):
         "combine_gbs": comb_bytes / (stage_avg["combine"] / 1e3) / 1e9,
         "hbm_peak_gbs": pk["hbm_gbs"],
         "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
+        "router_us": router_us,
     }
 
     cpu = None

@@ -24,10 +24,10 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
                 8: "MOE_ERR_BAD_INDEX"}
 
 EPI_STORE, EPI_SWIGLU, EPI_WEIGHT_SCATTER = 0, 1, 2
-OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED = 0, 1, 2, 3, 4
+OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE = 0, 1, 2, 3, 4, 5
 
 # Every symbol include/moe.h declares.
-EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_plan", "moe_dispatch",
+EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_plan", "moe_dispatch",
            "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
            "moe_last_error"]
@@ -61,6 +61,8 @@ def load(path: str | None = None):
     lib.moe_abi_version.restype = ctypes.c_int
     lib.moe_workspace_size.argtypes = [ctypes.c_int, i64, i64, i64, i32, i32]
     lib.moe_workspace_size.restype = sz
+    lib.moe_route.argtypes = [P, i64, i32, i32, P, P, P, sz, P]
+    lib.moe_route.restype = st
     lib.moe_plan.argtypes = [P, P, i64, i32, i32, P, P, P, P, P, P, sz, P]
     lib.moe_plan.restype = st
     lib.moe_dispatch.argtypes = [P, P, i64, i64, i32, P, P, sz, P]
@@ -117,6 +119,14 @@ def alloc_workspace(op: int, M: int, H: int, F: int, E: int, topk: int, device) 
     """A zeroed uint8 workspace of the size the op needs (torch allocations are 256-byte aligned)."""
     n = moe_workspace_size(op, M, H, F, E, topk)
     return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(logits, topk, topk_ids, topk_w, ws, stream=None):
+    M, E = logits.shape
+    if logits.dtype != torch.float32:
+        raise ValueError("moe_route takes fp32 logits")
+    _check(load().moe_route(_ptr(logits), M, E, topk, _ptr(topk_ids), _ptr(topk_w), _ptr(ws),
+                            ws.numel(), _stream(stream)))
 
 
 def moe_plan(topk_ids, topk_w, E, counts, offsets, perm, inv_perm, w_sorted, ws, stream=None):

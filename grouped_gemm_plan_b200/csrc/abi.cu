@@ -31,6 +31,8 @@ int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_
                      int32_t n_c, int32_t* status, void* sync_area, uint64_t timeout_ns,
                      int32_t withhold_mtile, int num_sms, cudaStream_t stream);
 int32_t profiled_n_c(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
+cudaError_t launch_route(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* ids,
+                         float* w, int num_sms, cudaStream_t stream);
 }  // namespace moe
 
 namespace {
@@ -197,6 +199,22 @@ moe_status moe_plan(const int32_t* topk_ids, const float* topk_w, int64_t M, int
                                      plan_scratch(ws), num_sms_current(),
                                      reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "moe_plan launch");
+  return MOE_OK;
+}
+
+moe_status moe_route(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* topk_ids,
+                     float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  st = check_ws(MOE_OP_ROUTE, ws, ws_bytes, M, 0, 0, E, topk);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "logits, topk_ids and topk_w must not be NULL");
+  cudaError_t err = moe::launch_route(logits, M, E, topk, topk_ids, topk_w, num_sms_current(),
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_route launch");
   return MOE_OK;
 }
 

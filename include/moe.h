@@ -86,7 +86,8 @@ typedef enum moe_op {
   MOE_OP_DISPATCH = 1,
   MOE_OP_GROUPED_GEMM = 2,
   MOE_OP_COMBINE = 3,
-  MOE_OP_FFN_FUSED = 4
+  MOE_OP_FFN_FUSED = 4,
+  MOE_OP_ROUTE = 5
 } moe_op;
 
 /* Version of this ABI (incremented on any incompatible change). */
@@ -99,6 +100,20 @@ int moe_abi_version(void);
  * should read 0 before the first call (zero the buffer once, or call
  * moe_get_device_status once, which clears it). */
 size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
+
+/*
+ * moe_route -- the router in front of the layer (the grouped GEMM article's
+ * introduction: the router hands each token to some experts; the pages define
+ * no more, so this is the plainest reading):
+ *   topk_ids[t, :] = the topk experts with the largest logits[t, :], largest
+ *                    first, ties to the lower expert index
+ *   topk_w[t, k]   = exp(l_k) / sum_j exp(l_j) over the chosen logits l_k
+ *   logits fp32 [M, E] (finite), topk_ids int32 [M, topk], topk_w fp32 [M, topk].
+ * Selection compares the given fp32 values exactly; the softmax runs in fp32.
+ * topk <= min(E, 32), E <= MOE_MAX_EXPERTS.
+ */
+moe_status moe_route(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* topk_ids,
+                     float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_plan -- routing plan ([PTO] "MegaMoE 融合算子七阶段", FrontReorder; [GG]

@@ -52,6 +52,8 @@ def configure(lib):
     lib.oracle_bruteforce_tokens.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P]
     lib.oracle_bruteforce_tokens.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_route.argtypes = [P, i64, i32, i32, P, P]
+    lib.oracle_route.restype = ctypes.c_int
     return lib
 
 
@@ -182,6 +184,19 @@ def moe_ffn(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
     if st != OK:
         raise OracleError(f"oracle_moe_ffn status {st}")
     return out
+
+
+def route(logits: np.ndarray, topk: int):
+    """Router: ids int32 [M, topk] (largest logits first, ties to the lower index) and
+    softmax weights fp64 [M, topk] over the chosen logits."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    M, E = logits.shape
+    ids = np.zeros((M, topk), np.int32)
+    w = np.zeros((M, topk), np.float64)
+    st = _load().oracle_route(_p(logits), M, E, topk, _p(ids), _p(w))
+    if st != OK:
+        raise OracleError(f"oracle_route status {st}")
+    return ids, w
 
 
 def bruteforce_tokens(x, W1, W2, ids: np.ndarray, w: np.ndarray, tokens) -> np.ndarray:

@@ -328,6 +328,49 @@ int oracle_bruteforce_tokens(const uint16_t *x, const uint16_t *W1, const uint16
     return ORACLE_OK;
 }
 
+/*
+ * Router (the step before the layer; the grouped GEMM article's introduction:
+ * the router hands each token to some experts).  Reading taken, since the pages
+ * define no router: a token goes to the topk experts with the largest logits,
+ * largest first, ties to the lower expert index; its gate weights are the
+ * softmax over those topk logits:
+ *   w[t, k] = exp(l[t, ids[t, k]]) / sum_j exp(l[t, ids[t, j]])
+ * Selection compares the given fp32 values exactly; the softmax runs in fp64
+ * (shifted by the largest chosen logit).  topk <= E; returns ORACLE_ERR_ARG
+ * otherwise.
+ */
+int oracle_route(const float *logits, int64_t M, int32_t E, int32_t topk, int32_t *ids,
+                 double *w)
+{
+    if (M < 0 || E < 1 || topk < 1 || topk > E)
+        return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < M; t++) {
+        const float *l = logits + t * E;
+        int32_t *out = ids + t * topk;
+        for (int32_t k = 0; k < topk; k++) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; e++) {
+                int taken = 0;
+                for (int32_t j = 0; j < k; j++)
+                    if (out[j] == e)
+                        taken = 1;
+                if (taken)
+                    continue;
+                if (best < 0 || l[e] > l[best])
+                    best = e;
+            }
+            out[k] = best;
+        }
+        double mx = (double)l[out[0]];
+        double sum = 0.0;
+        for (int32_t k = 0; k < topk; k++)
+            sum += exp((double)l[out[k]] - mx);
+        for (int32_t k = 0; k < topk; k++)
+            w[t * topk + k] = exp((double)l[out[k]] - mx) / sum;
+    }
+    return ORACLE_OK;
+}
+
 /* Number of OpenMP threads the oracle's parallel loops use. */
 int oracle_num_threads(void)
 {

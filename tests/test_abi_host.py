@@ -80,6 +80,15 @@ def test_plan_validation(lib):
     assert lib.moe_plan(FAKE, None, 4, 8, 2, FAKE, FAKE, FAKE, None, FAKE, FAKE_WS, 256, None) == 1
 
 
+def test_route_validation(lib):
+    r = lib.moe_route
+    assert r(FAKE, 4, 8, 9, FAKE, FAKE, FAKE_WS, 256, None) == 1        # topk > E
+    assert r(FAKE, 4, 64, 33, FAKE, FAKE, FAKE_WS, 256, None) == 2      # topk > 32
+    assert r(FAKE, 4, 2000, 2, FAKE, FAKE, FAKE_WS, 256, None) == 2     # E too large
+    assert r(None, 4, 8, 2, FAKE, FAKE, FAKE_WS, 256, None) == 1        # null logits
+    assert r(None, 0, 8, 2, None, None, FAKE_WS, 256, None) == 0        # M = 0: no-op
+
+
 def test_gemm_validation(lib):
     g = lib.moe_grouped_gemm
     ok = dict(E=8, R=256, K=256, N=512)

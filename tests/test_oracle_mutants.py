@@ -33,6 +33,9 @@ MUTANTS = {
                           "c[n] += a * bf16_widen(Be[(n % K) * N + (k % N)]);"),
     "w2_row_index": ("const uint16_t *wrow = W2e + j * H;",
                      "const uint16_t *wrow = W2e + (F - 1 - j) * H;"),
+    "route_tie_to_higher_index": ("if (best < 0 || l[e] > l[best])", "if (best < 0 || l[e] >= l[best])"),
+    "route_softmax_misses_shift": ("w[t * topk + k] = exp((double)l[out[k]] - mx) / sum;",
+                                   "w[t * topk + k] = exp((double)l[out[k]]) / sum;"),
     "tile_short_edge": ("tile_row1[n] = (r + BM < offsets[e + 1]) ? r + BM : offsets[e + 1];",
                         "tile_row1[n] = r + BM;"),
 }
@@ -55,6 +58,8 @@ CHILD = textwrap.dedent("""
         pins.test_scalar_closed_form_h1_f1,
         pins.test_identical_experts_sum_of_weights,
         pins.test_layer_matches_torch_per_token_mixture,
+        pins.test_route_matches_lexsort_and_softmax,
+        pins.test_route_closed_form_and_permutation_equivariance,
     ]
     caught = 0
     for c in calls:

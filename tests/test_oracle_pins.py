@@ -251,3 +251,42 @@ def test_layer_matches_torch_per_token_mixture():
             g = X[t] @ A[e]
             ref[t] += float(w[t, k]) * ((torch.nn.functional.silu(g[:F]) * g[F:]) @ B[e])
     np.testing.assert_allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- router
+
+def test_route_matches_lexsort_and_softmax():
+    rng = np.random.default_rng(21)
+    for M, E, k in [(50, 8, 2), (20, 64, 4), (9, 16, 16), (5, 1, 1)]:
+        logits = rng.standard_normal((M, E)).astype(np.float32)
+        logits[0, :] = 0.5                       # all tied: lowest indices first
+        ids, w = oracle.route(logits, k)
+        for t in range(M):
+            order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))[:k]
+            assert ids[t].tolist() == order.tolist()
+            chosen = logits[t, ids[t]].astype(np.float64)
+            ref = np.exp(chosen - chosen.max()) / np.exp(chosen - chosen.max()).sum()
+            np.testing.assert_allclose(w[t], ref, rtol=1e-14, atol=0)
+        assert ids[0].tolist() == list(range(k))
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+
+
+def test_route_closed_form_and_permutation_equivariance():
+    logits = np.array([[0.0, float(np.log(3.0)), -5.0]], np.float32)
+    ids, w = oracle.route(logits, 2)
+    assert ids.tolist() == [[1, 0]]
+    a = float(np.float32(np.log(3.0)))
+    np.testing.assert_allclose(w[0], [np.exp(a) / (np.exp(a) + 1), 1 / (np.exp(a) + 1)], rtol=1e-14)
+    # relabelling the experts relabels the choice and leaves the weights alone
+    rng = np.random.default_rng(22)
+    L = rng.standard_normal((30, 12)).astype(np.float32)   # distinct values: no ties
+    p = rng.permutation(12)
+    i1, w1 = oracle.route(L, 3)
+    i2, w2 = oracle.route(np.ascontiguousarray(L[:, p]), 3)
+    assert np.array_equal(p[i2], i1)
+    np.testing.assert_allclose(w2, w1, rtol=1e-15)
+
+
+def test_route_rejects_topk_above_e():
+    with pytest.raises(oracle.OracleError):
+        oracle.route(np.zeros((2, 3), np.float32), 4)
