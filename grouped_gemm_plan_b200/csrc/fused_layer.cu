@@ -5,8 +5,9 @@
 // This is the single-GPU analogue of COMET's thread-block specialisation (COMET
 // review, section 4.2.1): the first n_c CTAs are memory CTAs (dispatch, then
 // combine) and the rest are GEMM CTAs with the same warp-specialised tcgen05
-// pipeline as grouped_gemm.cu; the split n_c comes from profiled metadata
-// (section 4.2.2).  The hand-offs follow the shared-tensor decomposition of
+// pipeline as grouped_gemm.cu in warps 0-5, plus six memory warps (6-11) that do
+// the same dispatch and combine work in the GEMM SMs' idle issue slots; the split
+// n_c comes from profiled metadata (section 4.2.2).  The hand-offs follow the shared-tensor decomposition of
 // section 4.1.1: dispatch -> GEMM1 per m-tile (tokens are independent along M),
 // GEMM1 -> GEMM2 per m-tile once every GEMM1 column block of it is written, and
 // GEMM2 -> combine per token once all top-k rows of the token are complete (the
@@ -14,8 +15,8 @@
 // The PTO MegaMoE article describes the same idea with expert-level arrival and
 // ready flags instead of global barriers ("MegaMoE 融合算子七阶段").
 //
-// Work order.  Memory CTAs claim m-tiles for dispatch with an atomic counter in
-// the order GEMM1 consumes them; GEMM CTAs walk one static list: all GEMM1 tiles
+// Work order.  Memory warps claim dispatch items (16 rows of one m-tile) with an
+// atomic counter in the order GEMM1 consumes them; GEMM CTAs walk one static list: all GEMM1 tiles
 // (expert by expert, n-tile outer, m-tile inner) then all GEMM2 tiles.  Every
 // wait is on work that comes earlier in that order and all CTAs are co-resident
 // (cooperative launch, one CTA per SM), so the smallest unfinished item can
@@ -34,8 +35,11 @@ constexpr int L_BM = 128;
 constexpr int L_BN = 256;
 constexpr int L_BK = 64;
 constexpr int L_STAGES = 4;
-constexpr int L_THREADS = 192;
+constexpr int L_THREADS = 384;          // 6 GEMM-role warps + 6 memory warps
 constexpr int L_WARPS = L_THREADS / 32;
+constexpr int L_FIRST_MEM_WARP = 6;      // in GEMM CTAs, warps 6..11 do memory work
+constexpr int L_GROUP_ROWS = 16;         // rows of one dispatch work item
+constexpr int L_GROUPS_PER_MT = 128 / L_GROUP_ROWS;
 constexpr int L_A_BYTES = L_BM * L_BK * 2;
 constexpr int L_B_BOX_BYTES = L_BK * 64 * 2;
 constexpr int L_STAGE_BYTES = L_A_BYTES + 4 * L_B_BOX_BYTES;
@@ -49,10 +53,10 @@ constexpr uint32_t L_IDESC = idesc_bf16_f32(L_BM, L_BN, true);
 struct LayerSync {
   int32_t* abort;          // [1] any CTA gave up
   int32_t* progress;       // [1] completed work items (tiles, dispatched m-tiles, tokens)
-  int32_t* dispatch_head;  // [1] next m-tile to dispatch
+  int32_t* dispatch_head;  // [1] next dispatch item (m-tile, group of 16 rows)
   int32_t* combine_head;   // [1] next slot of the ready list to combine
   int32_t* ready_tail;     // [1] next free slot of the ready list
-  int32_t* xp_ready;       // [MT] 1 once the m-tile's rows of Xp are written
+  int32_t* xp_ready;       // [MT] groups of 16 rows of the m-tile written to Xp
   int32_t* h_done;         // [MT] GEMM1 warps that wrote their rows of h (4 per n-tile)
   int32_t* row_done;       // [R] GEMM2 column tiles written for the row
   int32_t* tok_done;       // [M] complete rows of the token
@@ -108,8 +112,9 @@ __device__ __forceinline__ LTile decode(int32_t t, int32_t nt, const int32_t* s_
 // Wait until *flag >= target.  Gives up (false) when the global abort flag is
 // raised or when the progress counter has not moved for timeout_ns.
 __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t target, const LayerSync& sy,
-                                          uint64_t timeout_ns) {
+                                          uint64_t timeout_ns, uint32_t max_sleep_ns = 128) {
   if (ld_acquire(flag) >= target) return true;
+  uint32_t sleep_ns = 32;
   int32_t last = ld_relaxed(sy.progress);
   uint64_t t0 = globaltimer_ns();
   for (;;) {
@@ -123,7 +128,8 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t target, c
     } else if (now - t0 > timeout_ns) {
       return false;
     }
-    __nanosleep(128);
+    __nanosleep(sleep_ns);
+    if (sleep_ns < max_sleep_ns) sleep_ns *= 2;
   }
 }
 
@@ -157,6 +163,100 @@ __device__ __forceinline__ void give_up(const LayerArgs& a, volatile int32_t* sa
   *sabort = 1;
 }
 
+// Memory work of one warp: first dispatch items (16 rows of one m-tile, in
+// GEMM1's order; the warp that completes a group counts it on the m-tile), then
+// combine tokens from the ready list as GEMM2 completes them.  Runs in every warp
+// of a memory CTA and in warps 6..11 of every GEMM CTA.
+__device__ void memory_warp(const LayerArgs& a, const int32_t* s_ms, const int32_t* s_off,
+                            int32_t E, int32_t MT, volatile int32_t* s_abort, int lane) {
+  const LayerSync& sy = a.sync;
+  const int32_t vpr = a.H / 8;  // 16-byte vectors per bf16 row
+  // ---- dispatch
+  for (;;) {
+    int32_t item = 0;
+    if (lane == 0) item = ld_relaxed(sy.abort) != 0 ? MT * L_GROUPS_PER_MT : atomicAdd(sy.dispatch_head, 1);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    const int32_t mt = item / L_GROUPS_PER_MT;
+    if (mt >= MT) break;
+    const int32_t grp = item - mt * L_GROUPS_PER_MT;
+    int32_t lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int32_t mid = (lo + hi) >> 1;
+      if (s_ms[mid] <= mt) lo = mid; else hi = mid;
+    }
+    const int32_t row0 = s_off[lo] + (mt - s_ms[lo]) * L_BM;
+    const int32_t rows = min(L_BM, s_off[lo + 1] - row0);
+    const int32_t r0 = grp * L_GROUP_ROWS;
+    if (r0 >= rows) continue;  // the m-tile is short: this group has no rows
+    const int32_t r1 = min(r0 + L_GROUP_ROWS, rows);
+    for (int32_t r = r0; r < r1; ++r) {
+      const int32_t s = row0 + r;
+      const int32_t i = __ldg(a.perm + s);
+      uint4* dst = a.xp + static_cast<int64_t>(s) * vpr;
+      if (i < 0 || i >= a.R) {
+        if (lane == 0) set_status(a.status, MOE_ERR_BAD_INDEX);
+        for (int32_t c = lane; c < vpr; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      const uint4* src = a.x + static_cast<int64_t>(i / a.topk) * vpr;
+      int32_t c = lane;
+      for (; c + 96 < vpr; c += 128) {
+        const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32), v2 = __ldg(src + c + 64),
+                    v3 = __ldg(src + c + 96);
+        dst[c] = v0;
+        dst[c + 32] = v1;
+        dst[c + 64] = v2;
+        dst[c + 96] = v3;
+      }
+      for (; c < vpr; c += 32) dst[c] = __ldg(src + c);
+    }
+    __syncwarp();
+    if (lane == 0 && mt != a.withhold_mtile) {
+      __threadfence();
+      fence_proxy_async_global();  // the rows are read next by TMA (async proxy)
+      red_release_add(sy.xp_ready + mt, 1);
+      red_release_add(sy.progress, 1);
+    }
+  }
+  // ---- combine, token by token as tokens complete
+  const int32_t steps = (vpr + 31) / 32;
+  for (;;) {
+    int32_t idx = 0;
+    if (lane == 0) idx = atomicAdd(sy.combine_head, 1);
+    idx = __shfl_sync(0xffffffffu, idx, 0);
+    if (idx >= a.M) break;
+    int32_t v = 0;
+    if (lane == 0)
+      v = wait_flag(sy.ready_list + idx, 1, sy, a.timeout_ns, 2048) ? ld_acquire(sy.ready_list + idx)
+                                                                    : 0;
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v <= 0) {
+      if (lane == 0 && ld_relaxed(sy.abort) == 0) give_up(a, s_abort);
+      break;
+    }
+    const int32_t t = v - 1;
+    const float4* yrow = reinterpret_cast<const float4*>(a.yk) + static_cast<int64_t>(t) * a.topk * (a.H / 4);
+    for (int32_t q = 0; q < steps; ++q) {
+      const int32_t c = q * 32 + lane;  // group of 8 columns
+      if (c >= vpr) break;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int32_t k = 0; k < a.topk; ++k) {
+        const float4* p = yrow + static_cast<int64_t>(k) * (a.H / 4) + 2 * c;
+        const float4 u0 = __ldcg(p), u1 = __ldcg(p + 1);
+        acc[0] += u0.x; acc[1] += u0.y; acc[2] += u0.z; acc[3] += u0.w;
+        acc[4] += u1.x; acc[5] += u1.y; acc[6] += u1.z; acc[7] += u1.w;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      a.out[static_cast<int64_t>(t) * vpr + c] = o;
+    }
+    if (lane == 0) red_release_add(sy.progress, 1);
+  }
+}
+
 __global__ void __launch_bounds__(L_THREADS, 1)
     moe_layer_kernel(const __grid_constant__ CUtensorMap tmXp,
                      const __grid_constant__ CUtensorMap tmW1,
@@ -170,7 +270,6 @@ __global__ void __launch_bounds__(L_THREADS, 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int32_t s_abort;
-  __shared__ int32_t s_claim;
   __shared__ int32_t s_plan_ok;
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_ms[MOE_MAX_EXPERTS + 1];
@@ -241,87 +340,7 @@ __global__ void __launch_bounds__(L_THREADS, 1)
 
   if (memory_cta) {
     // ================================================================ memory CTA
-    if (!s_plan_ok) return;       // a failed plan: nothing to dispatch or combine
-    const int32_t vpr = a.H / 8;  // 16-byte vectors per bf16 row
-    // ---- dispatch, m-tile by m-tile, in GEMM1's order
-    for (;;) {
-      // one thread decides for the block, so every thread leaves the loop together
-      if (tid == 0) s_claim = ld_relaxed(sy.abort) != 0 ? MT : atomicAdd(sy.dispatch_head, 1);
-      __syncthreads();
-      const int32_t mt = s_claim;
-      __syncthreads();
-      if (mt >= MT) break;
-      int32_t lo = 0, hi = E;
-      while (hi - lo > 1) {
-        const int32_t mid = (lo + hi) >> 1;
-        if (s_ms[mid] <= mt) lo = mid; else hi = mid;
-      }
-      const int32_t row0 = s_off[lo] + (mt - s_ms[lo]) * L_BM;
-      const int32_t rows = min(L_BM, s_off[lo + 1] - row0);
-      for (int32_t r = warp; r < rows; r += L_WARPS) {
-        const int32_t s = row0 + r;
-        const int32_t i = __ldg(a.perm + s);
-        uint4* dst = a.xp + static_cast<int64_t>(s) * vpr;
-        if (i < 0 || i >= a.R) {
-          if (lane == 0) set_status(a.status, MOE_ERR_BAD_INDEX);
-          for (int32_t c = lane; c < vpr; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
-          continue;
-        }
-        const uint4* src = a.x + static_cast<int64_t>(i / a.topk) * vpr;
-        int32_t c = lane;
-        for (; c + 96 < vpr; c += 128) {
-          const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32), v2 = __ldg(src + c + 64),
-                      v3 = __ldg(src + c + 96);
-          dst[c] = v0;
-          dst[c + 32] = v1;
-          dst[c + 64] = v2;
-          dst[c + 96] = v3;
-        }
-        for (; c < vpr; c += 32) dst[c] = __ldg(src + c);
-      }
-      __syncthreads();
-      if (tid == 0 && mt != a.withhold_mtile) {
-        __threadfence();
-        fence_proxy_async_global();  // the rows are read next by TMA (async proxy)
-        st_release(sy.xp_ready + mt, 1);
-        red_release_add(sy.progress, 1);
-      }
-    }
-    // ---- combine, token by token as tokens complete
-    const int32_t steps = (vpr + 31) / 32;
-    for (;;) {
-      int32_t idx = 0;
-      if (lane == 0) idx = atomicAdd(sy.combine_head, 1);
-      idx = __shfl_sync(0xffffffffu, idx, 0);
-      if (idx >= a.M) break;
-      int32_t v = 0;
-      if (lane == 0) v = wait_flag(sy.ready_list + idx, 1, sy, a.timeout_ns) ? ld_acquire(sy.ready_list + idx) : 0;
-      v = __shfl_sync(0xffffffffu, v, 0);
-      if (v <= 0) {
-        if (lane == 0 && ld_relaxed(sy.abort) == 0) give_up(a, &s_abort);
-        break;
-      }
-      const int32_t t = v - 1;
-      const float4* yrow = reinterpret_cast<const float4*>(a.yk) + static_cast<int64_t>(t) * a.topk * (a.H / 4);
-      for (int32_t q = 0; q < steps; ++q) {
-        const int32_t c = q * 32 + lane;  // group of 8 columns
-        if (c >= vpr) break;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int32_t k = 0; k < a.topk; ++k) {
-          const float4* p = yrow + static_cast<int64_t>(k) * (a.H / 4) + 2 * c;
-          const float4 u0 = __ldcg(p), u1 = __ldcg(p + 1);
-          acc[0] += u0.x; acc[1] += u0.y; acc[2] += u0.z; acc[3] += u0.w;
-          acc[4] += u1.x; acc[5] += u1.y; acc[6] += u1.z; acc[7] += u1.w;
-        }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        a.out[static_cast<int64_t>(t) * vpr + c] = o;
-      }
-      if (lane == 0) red_release_add(sy.progress, 1);
-    }
+    if (s_plan_ok) memory_warp(a, s_ms, s_off, E, MT, &s_abort, lane);
     return;  // no TMEM, no outstanding async copies
   }
 
@@ -339,7 +358,8 @@ __global__ void __launch_bounds__(L_THREADS, 1)
       const bool two = t >= T1;
       const LTile tc = two ? decode(t - T1, a.nt2, s_ms, s_off, E) : decode(t, a.nt1, s_ms, s_off, E);
       const bool ok = two ? wait_flag(sy.h_done + tc.mt, 4 * a.nt1, sy, a.timeout_ns)
-                          : wait_flag(sy.xp_ready + tc.mt, 1, sy, a.timeout_ns);
+                          : wait_flag(sy.xp_ready + tc.mt, (tc.rows + L_GROUP_ROWS - 1) / L_GROUP_ROWS,
+                                      sy, a.timeout_ns);
       if (!ok) {
         give_up(a, &s_abort);
         break;
@@ -428,6 +448,9 @@ __global__ void __launch_bounds__(L_THREADS, 1)
       umma_commit(&drain_bar);
       mbar_wait_bounded(&drain_bar, 0, a.timeout_ns, nullptr);
     }
+  } else if (warp >= L_FIRST_MEM_WARP) {
+    // ------------------------------------------------------------ memory warps
+    if (s_plan_ok) memory_warp(a, s_ms, s_off, E, MT, &s_abort, lane);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;

@@ -191,8 +191,9 @@ moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
  *   n_c: thread blocks given to the memory stages (dispatch / combine) while the
  *   GEMM blocks run, [COMET] 4.2.1-4.2.2.  0 runs the stages as consecutive
  *   kernels; n_c >= 1 runs plan, then ONE persistent cooperative kernel with one
- *   CTA per SM, of which n_c dispatch and combine while the rest run the GEMM
- *   tiles, handing off through per-m-tile and per-token ready flags;
+ *   CTA per SM, of which n_c only dispatch and combine while the rest run the
+ *   GEMM tiles with six further memory warps each, handing off through
+ *   per-m-tile and per-token ready counters;
  *   -1 takes the value from the library's profiled table for this shape.
  *   n_c must be below 65 and below the SM count.
  * H and F must be multiples of 64.
