@@ -405,16 +405,18 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
                             const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                             int num_sms, cudaStream_t stream);
 
-// Which kernel runs a grouped GEMM: the single-CTA kernel (128-row tiles) unless
-// MOE_GEMM_PAIR=1 in the environment selects the CTA-pair kernel (256-row tiles);
-// the tests run both.
+// Which kernel runs a grouped GEMM.  The CTA-pair kernel (256-row tiles) moves a
+// third fewer bytes into each SM per MMA and wins once experts hold many rows;
+// with fewer rows per expert its 256-row tiles pad more rows than the
+// single-CTA kernel's 128-row tiles and it loses.  Measured on B200: pair faster
+// at 1024 and 2048 rows per expert (Mixtral and Phi-3.5 shapes), slower at 512
+// and 256 (Qwen2 and wide M=512 shapes).  MOE_GEMM_PAIR=0/1 in the environment
+// forces one kernel (the tests run both).
 static bool use_pair_kernel(int64_t R, int32_t E) {
   const char* v = getenv("MOE_GEMM_PAIR");
   if (v != nullptr && v[0] == '0') return false;
   if (v != nullptr && v[0] == '1') return true;
-  (void)R;
-  (void)E;
-  return false;  // measured slower than the single-CTA kernel on every workload so far
+  return E > 0 && R >= 1024 * static_cast<int64_t>(E);
 }
 
 static int launch_grouped_gemm_1sm(const void* A, const void* B, const int32_t* offsets, int32_t E,

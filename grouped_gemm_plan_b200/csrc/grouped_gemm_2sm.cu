@@ -8,8 +8,10 @@
 // 128 rows of A and one half (128 columns) of B, and the leader CTA issues one
 // M = 256, N = 256 MMA that reads A and B from both CTAs' shared memory and
 // writes each CTA's 128 rows of the accumulator into that CTA's TMEM.  Per SM
-// that halves the B bytes fetched for the same work, and with 32 KB per stage
-// six stages fit where four did.
+// that halves the B bytes fetched for the same work (32 KB per 64 of K instead
+// of 48 KB).  A stage holds 128 of K (eight MMAs per barrier round trip, three
+// 64 KB stages), since the pair's barrier hand-offs cross SMs and cost more per
+// round trip than the single-CTA kernel's.
 //
 // Protocol (leader = cluster rank 0, peer = rank 1):
 //   full[s]    leader's barrier; the leader arrives with the byte count of both
@@ -27,11 +29,12 @@ namespace {
 
 constexpr int P_BM = 256;                 // rows per CTA pair
 constexpr int P_BN = 256;
-constexpr int P_BK = 64;
-constexpr int P_STAGES = 6;
+constexpr int P_BK = 128;                 // K per stage: 8 MMAs per barrier round trip
+constexpr int P_STAGES = 3;
 constexpr int P_THREADS = 192;
-constexpr int P_A_BYTES = 128 * P_BK * 2;       // this CTA's 128 rows
-constexpr int P_B_BOX_BYTES = P_BK * 64 * 2;
+constexpr int P_A_BOX_BYTES = 128 * 64 * 2;     // 128 rows x 64 K (one 128-byte swizzle span)
+constexpr int P_A_BYTES = (P_BK / 64) * P_A_BOX_BYTES;  // this CTA's 128 rows
+constexpr int P_B_BOX_BYTES = P_BK * 64 * 2;    // 64 columns x P_BK rows of K
 constexpr int P_B_BYTES = 2 * P_B_BOX_BYTES;    // this CTA's 128 columns
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_TMEM_COLS = 512;
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
 
   const uint32_t tmem_base = s_tmem_base;
   const int32_t T = s_tstart[E];
-  const int32_t KB = args.K / P_BK;
+  const int32_t KB = (args.K + P_BK - 1) / P_BK;  // a short last k-block reads zeros
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -283,7 +286,9 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         }
         uint8_t* sa = ring + stage * P_STAGE_BYTES;
         uint8_t* sb = sa + P_A_BYTES;
-        tma2_load_2d(sa, &tmA, fb, kb * P_BK, arow);
+#pragma unroll
+        for (int c = 0; c < P_BK / 64; ++c)
+          tma2_load_2d(sa + c * P_A_BOX_BYTES, &tmA, fb, kb * P_BK + 64 * c, arow);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           int32_t n;
@@ -329,8 +334,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         const uint32_t b_addr = a_addr + P_A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < P_BK / 16; ++kk) {
-          const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
+          const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * P_A_BOX_BYTES + (kk & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, P_B_BOX_BYTES, 1024);
           umma2_bf16(d_tmem, adesc, bdesc, P_IDESC, (kb | kk) != 0 ? 1u : 0u);
         }
         issued_any = true;
@@ -482,7 +487,7 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
   const cuuint64_t bdims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
                                static_cast<cuuint64_t>(E)};
   const cuuint64_t bstr[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(K * N) * 2};
-  const cuuint32_t bbox[3] = {64, 64, 1};
+  const cuuint32_t bbox[3] = {64, P_BK, 1};
   if (!enc2(&tmA, 2, A, adims, astr, abox) || !enc2(&tmB, 3, B, bdims, bstr, bbox)) return 1;
   Gemm2Args a;
   a.offsets = offsets;
