@@ -30,7 +30,7 @@ OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE = 0, 1
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_plan", "moe_dispatch",
            "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
-           "moe_last_error"]
+           "moe_set_stage_events", "moe_last_error"]
 
 
 class MoEError(RuntimeError):
@@ -81,6 +81,8 @@ def load(path: str | None = None):
     lib.moe_set_wait_timeout_ns.restype = None
     lib.moe_set_fault_injection.argtypes = [i32, i32]
     lib.moe_set_fault_injection.restype = st
+    lib.moe_set_stage_events.argtypes = [P]
+    lib.moe_set_stage_events.restype = st
     lib.moe_last_error.restype = ctypes.c_char_p
     if path is None:
         _lib = lib
@@ -195,6 +197,22 @@ def moe_set_wait_timeout_ns(ns: int) -> None:
 def moe_set_fault_injection(kind: int, index: int = 0) -> None:
     """Test hook (see include/moe.h): 1 = withhold one m-tile's dispatch flag, 0 = off."""
     _check(load().moe_set_fault_injection(int(kind), int(index)))
+
+
+def moe_set_stage_events(events) -> None:
+    """Stage timing of moe_ffn_fused (see include/moe.h): `events` is None (off) or
+    six torch.cuda.Event(enable_timing=True); each is recorded once here so that its
+    CUDA event exists.  The caller keeps the events alive while they are set."""
+    if events is None:
+        _check(load().moe_set_stage_events(None))
+        return
+    if len(events) != 6:
+        raise ValueError("moe_set_stage_events takes six events")
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(load().moe_set_stage_events(arr))
 
 
 def moe_last_error() -> str:

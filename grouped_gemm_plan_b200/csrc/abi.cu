@@ -40,6 +40,13 @@ namespace {
 thread_local std::string g_last_error;
 uint64_t g_timeout_ns = 2000000000ull;
 int32_t g_withhold_mtile = -1;  // fault injection for tests (moe_set_fault_injection)
+thread_local cudaEvent_t g_stage_events[6];  // moe_set_stage_events
+thread_local bool g_stage_events_on = false;
+
+// Records stage event i of moe_ffn_fused when stage timing is on.
+void stage_mark(int i, cudaStream_t s) {
+  if (g_stage_events_on) cudaEventRecord(g_stage_events[i], s);
+}
 
 constexpr size_t kCtrlBytes = 256;
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
@@ -149,6 +156,17 @@ int moe_abi_version(void) { return 1; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns > 0 ? ns : 1; }
+
+moe_status moe_set_stage_events(void* const* events) {
+  g_last_error.clear();
+  if (events == nullptr) {
+    g_stage_events_on = false;
+    return MOE_OK;
+  }
+  for (int i = 0; i < 6; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_stage_events_on = true;
+  return MOE_OK;
+}
 
 moe_status moe_set_fault_injection(int32_t kind, int32_t index) {
   if (kind == 0) {
@@ -331,9 +349,11 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
   const int sms = num_sms_current();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
+  stage_mark(0, s);
   cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
                                      perm, nullptr, w_sorted, status, plan_scratch(ws), sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused plan");
+  stage_mark(1, s);
   const int32_t nc = n_c < 0 ? moe::profiled_n_c(M, H, F, E, topk) : n_c;
   if (nc > 0) {
     // One persistent kernel: nc memory CTAs (dispatch, combine) beside the GEMM CTAs.
@@ -344,20 +364,25 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     if (rc == 1) return fail(MOE_ERR_CUDA, "tensor map encode failed (layer kernel)");
     if (rc == 3) return fail(MOE_ERR_CUDA, "cooperative launch refused: the layer kernel needs one co-resident CTA per SM");
     if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_ffn_fused layer kernel");
+    for (int i = 2; i <= 5; ++i) stage_mark(i, s);
     return MOE_OK;
   }
   err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused dispatch");
+  stage_mark(2, s);
   int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,
                                     nullptr, h, status, g_timeout_ns, sms, s);
   if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM1)")
                               : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM1");
+  stage_mark(3, s);
   rc = moe::launch_grouped_gemm(h, W2, offsets, E, R, F, H, MOE_EPI_WEIGHT_SCATTER, w_sorted, perm,
                                 yk, status, g_timeout_ns, sms, s);
   if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM2)")
                               : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM2");
+  stage_mark(4, s);
   err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused combine");
+  stage_mark(5, s);
   return MOE_OK;
 }
 

@@ -262,6 +262,19 @@ void moe_set_wait_timeout_ns(uint64_t ns);
  * Process-wide; returns MOE_ERR_INVALID_ARG for an unknown kind. */
 moe_status moe_set_fault_injection(int32_t kind, int32_t index);
 
+/* Stage timing for moe_ffn_fused (measurement only; the pages have no
+ * counterpart).  events: NULL (off, the default) or an array of 6 cudaEvent_t
+ * handles created by the caller; the caller keeps ownership and must keep them
+ * alive while set.  While set, each moe_ffn_fused call on this thread records
+ * events[0] on its stream before the plan and events[i + 1] after stage i
+ * (plan, dispatch, GEMM1 + SwiGLU, GEMM2 + scatter, combine), so that the
+ * elapsed time between consecutive events is one stage's device time.  In the
+ * single-kernel layer (n_c > 0) events[2..5] are all recorded after the layer
+ * kernel.  Recording an event between two kernels serialises them, so a
+ * programmatic dependent launch between those kernels no longer overlaps.
+ * Thread-local; returns MOE_OK. */
+moe_status moe_set_stage_events(void* const* events);
+
 /* Message of the last host-side error on this thread ("" if none). */
 const char* moe_last_error(void);
 

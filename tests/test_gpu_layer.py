@@ -138,6 +138,35 @@ def test_layer_deterministic(cuda_dev):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("n_c", [0, 2])
+def test_stage_events(cuda_dev, n_c):
+    """moe_set_stage_events: six events around the stages of one call, in order, the
+    stage times summing to the call's time; the output is unchanged by timing."""
+    w, x, W1, W2, ids, tw = layer_case(700, 512, 384, 8, 2, "skewed", seed=21)
+    ref = run_fused(cuda_dev, x, W1, W2, ids, tw, n_c=n_c)[0]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    B.moe_set_stage_events(evs)
+    try:
+        outer[0].record()
+        got = run_fused(cuda_dev, x, W1, W2, ids, tw, n_c=n_c)[0]
+        outer[1].record()
+    finally:
+        B.moe_set_stage_events(None)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    stages = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]
+    assert all(t >= 0.0 for t in stages), stages
+    assert stages[2] > 0.0 and stages[3] > 0.0 or n_c > 0
+    total = evs[0].elapsed_time(evs[5])
+    assert abs(sum(stages) - total) < 1e-3 + 1e-3 * total
+    assert total <= outer[0].elapsed_time(outer[1]) + 1e-3
+    # off again: a later call records nothing (the events keep their times)
+    run_fused(cuda_dev, x, W1, W2, ids, tw, n_c=n_c)
+    torch.cuda.synchronize()
+    assert evs[0].elapsed_time(evs[5]) == total
+
+
 def _sample_tokens(ids, n, seed):
     """First, last and random tokens, plus one token of the heaviest and lightest expert."""
     M = ids.shape[0]
