@@ -36,7 +36,6 @@ constexpr int L_BN = 256;
 constexpr int L_BK = 64;
 constexpr int L_STAGES = 4;
 constexpr int L_THREADS = 384;          // 6 GEMM-role warps + 6 memory warps
-constexpr int L_WARPS = L_THREADS / 32;
 constexpr int L_FIRST_MEM_WARP = 6;      // in GEMM CTAs, warps 6..11 do memory work
 constexpr int L_GROUP_ROWS = 16;         // rows of one dispatch work item
 constexpr int L_GROUPS_PER_MT = 128 / L_GROUP_ROWS;
