@@ -54,6 +54,15 @@ def configure(lib):
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_route.argtypes = [P, i64, i32, i32, P, P]
     lib.oracle_route.restype = ctypes.c_int
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_quantize_rows_e4m3.argtypes = [P, i64, i64, P, P]
+    lib.oracle_quantize_cols_e4m3.argtypes = [P, i32, i64, i64, P, P]
+    lib.oracle_grouped_gemm_e4m3.argtypes = [P, P, P, P, P, i32, i64, i64, P]
+    lib.oracle_moe_ffn_fp8.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P]
+    lib.oracle_moe_ffn_fp8.restype = ctypes.c_int
     return lib
 
 
@@ -214,4 +223,73 @@ def bruteforce_tokens(x, W1, W2, ids: np.ndarray, w: np.ndarray, tokens) -> np.n
                                           topk, _p(tok), tok.size, _p(out))
     if st != OK:
         raise OracleError(f"oracle_bruteforce_tokens status {st}")
+    return out
+
+
+# ------------------------------------------------------------------ FP8 (E4M3)
+
+def e4m3_decode(codes) -> np.ndarray:
+    """fp64 values of E4M3 codes (uint8 array)."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_decode(int(v)) for v in c.reshape(-1)]).reshape(c.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """E4M3 codes of float32 values (nearest, ties to even, saturating at 448)."""
+    lib = _load()
+    v = np.asarray(values, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_encode(float(x)) for x in v.reshape(-1)],
+                    dtype=np.uint8).reshape(v.shape)
+
+
+def quantize_rows_e4m3(A):
+    """Per-row E4M3 quantisation of bf16 A [R, K] -> (codes uint8 [R, K], scale fp32 [R])."""
+    a = _u16(A)
+    R, K = a.shape
+    q = np.empty((R, K), np.uint8)
+    sc = np.empty(R, np.float32)
+    _load().oracle_quantize_rows_e4m3(_p(a), R, K, _p(q), _p(sc))
+    return q, sc
+
+
+def quantize_cols_e4m3(B):
+    """Per-output-column E4M3 quantisation of bf16 B [E, K, N] -> (codes uint8 [E, N, K]
+    with K contiguous, scale fp32 [E, N])."""
+    b = _u16(B)
+    E, K, N = b.shape
+    q = np.empty((E, N, K), np.uint8)
+    sc = np.empty((E, N), np.float32)
+    _load().oracle_quantize_cols_e4m3(_p(b), E, K, N, _p(q), _p(sc))
+    return q, sc
+
+
+def grouped_gemm_e4m3(Aq, a_scale, BqT, b_scale, offsets) -> np.ndarray:
+    """fp64 C [R, N] = a_scale[s] * b_scale[e, n] * (decode(Aq[s]) . decode(BqT[e, n]))."""
+    Aq = np.ascontiguousarray(Aq, np.uint8)
+    BqT = np.ascontiguousarray(BqT, np.uint8)
+    a_scale = np.ascontiguousarray(a_scale, np.float32)
+    b_scale = np.ascontiguousarray(b_scale, np.float32)
+    offsets = np.ascontiguousarray(offsets, np.int32)
+    R, K = Aq.shape
+    E, N, _ = BqT.shape
+    C = np.zeros((R, N), np.float64)
+    _load().oracle_grouped_gemm_e4m3(_p(Aq), _p(a_scale), _p(BqT), _p(b_scale), _p(offsets), E,
+                                     K, N, _p(C))
+    return C
+
+
+def moe_ffn_fp8(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The layer with an E4M3 down projection (h and W2 quantised as above), fp64 [M, H]."""
+    xu, w1u, w2u = _u16(x), _u16(W1), _u16(W2)
+    M, H = xu.shape
+    E, _, F2 = w1u.shape
+    ids = np.ascontiguousarray(ids, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    topk = ids.shape[1]
+    out = np.zeros((M, H), np.float64)
+    st = _load().oracle_moe_ffn_fp8(_p(xu), _p(w1u), _p(w2u), _p(ids), _p(w), M, H, F2 // 2, E,
+                                    topk, _p(out))
+    if st != OK:
+        raise ValueError(f"oracle_moe_ffn_fp8 status {st}")
     return out

@@ -39,6 +39,13 @@
  *                   H=F=1 closed form; identical experts => out = FFN(x) * sum w;
  *                   linearity in w; per-token brute force equals the plan path
  *                   bit-exactly
+ *   e4m3 codec      torch.float8_e4m3fn on every code and on rounding ties;
+ *                   brute-force nearest grid value
+ *   fp8 quantisers  torch fp32 division + torch e4m3 conversion; round trip
+ *                   within half a grid step; the largest element maps to 448
+ *   fp8 GEMM        numpy float64 matmul of the decoded operands
+ *   fp8 layer       E=1,topk=1 equals torch's dense chain with the same
+ *                   quantisation; within the e4m3 error bound of the exact layer
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -372,6 +379,242 @@ int oracle_route(const float *logits, int64_t M, int32_t E, int32_t topk, int32_
 }
 
 /* Number of OpenMP threads the oracle's parallel loops use. */
+/* ------------------------------------------------------------------ FP8 (E4M3) */
+
+/*
+ * 8-bit floating point E4M3 (the OCP 8-bit format without infinities): bit 7
+ * sign, bits 6..3 exponent with bias 7, bits 2..0 mantissa.  Exponent field 0 is
+ * subnormal: value = m * 2^-9.  Otherwise value = (1 + m/8) * 2^(exp - 7).  The
+ * pattern S.1111.111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.
+ */
+double oracle_e4m3_decode(uint8_t c)
+{
+    int sign = c >> 7, ex = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (ex == 15 && m == 7)
+        return NAN;
+    if (ex == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, ex - 7);
+    return sign ? -v : v;
+}
+
+/*
+ * Nearest E4M3 value to v, ties to the even mantissa; magnitudes that round
+ * beyond 448 saturate to 448 (the conversion the quantiser uses); NaN -> 0x7F.
+ * Every step is exact in fp64: |v| is a float, the grid spacing a power of two.
+ */
+uint8_t oracle_e4m3_encode(float v)
+{
+    if (isnan(v))
+        return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs((double)v);
+    /* spacing of the grid around a: 2^(e-3) in binade [2^e, 2^(e+1)), e >= -6;
+       the subnormal range [0, 2^-6) has spacing 2^-9 */
+    int e = -6;
+    if (a >= ldexp(1.0, -6)) {
+        int ex;
+        frexp(a, &ex); /* a = f * 2^ex with f in [0.5, 1) */
+        e = ex - 1;
+    }
+    double step = ldexp(1.0, e - 3);
+    double q = a / step; /* exact: division by a power of two */
+    double fl = floor(q);
+    double rem = q - fl;
+    double n = fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0))
+        n = fl + 1.0;
+    double r = n * step; /* rounded magnitude */
+    if (r > 448.0)
+        r = 448.0;
+    if (r < ldexp(1.0, -6))
+        return sign | (uint8_t)(r / ldexp(1.0, -9)); /* subnormal (or zero) */
+    int ex;
+    double f = frexp(r, &ex); /* r = f * 2^ex, f in [0.5, 1) */
+    int be = ex - 1 + 7;     /* biased exponent */
+    int m = (int)((f * 2.0 - 1.0) * 8.0);
+    return sign | (uint8_t)(be << 3) | (uint8_t)m;
+}
+
+/*
+ * Per-row scaled quantisation of a bf16 matrix A [R, K] (the SwiGLU output h):
+ *   scale[r] = max_k |A[r, k]| / 448   (fp32 division; 1 for an all-zero row)
+ *   q[r, k]  = e4m3(A[r, k] / scale[r]) (fp32 division, then the encoding above)
+ * so that A[r, k] ~= scale[r] * decode(q[r, k]) and the largest element maps to
+ * +-448.  This is the "quantise right after SwiGLU" step of the PTO MegaMoE
+ * article (section "MegaMoE 融合算子七阶段"), with one scale per row (token).
+ */
+void oracle_quantize_rows_e4m3(const uint16_t *A, int64_t R, int64_t K, uint8_t *q, float *scale)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float v = fabsf((float)bf16_widen(A[r * K + k]));
+            if (v > amax)
+                amax = v;
+        }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = sc;
+        for (int64_t k = 0; k < K; k++)
+            q[r * K + k] = oracle_e4m3_encode((float)bf16_widen(A[r * K + k]) / sc);
+    }
+}
+
+/*
+ * Per-output-column scaled quantisation of bf16 weights B [E, K, N] (row-major, N
+ * contiguous), written transposed so that K is contiguous:
+ *   scale[e, n] = max_k |B[e, k, n]| / 448   (1 for an all-zero column)
+ *   qT[e, n, k] = e4m3(B[e, k, n] / scale[e, n])
+ */
+void oracle_quantize_cols_e4m3(const uint16_t *B, int32_t E, int64_t K, int64_t N, uint8_t *qT,
+                               float *scale)
+{
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *Be = B + (int64_t)e * K * N;
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; n++) {
+            float amax = 0.0f;
+            for (int64_t k = 0; k < K; k++) {
+                float v = fabsf((float)bf16_widen(Be[k * N + n]));
+                if (v > amax)
+                    amax = v;
+            }
+            float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+            scale[(int64_t)e * N + n] = sc;
+            uint8_t *qrow = qT + ((int64_t)e * N + n) * K;
+            for (int64_t k = 0; k < K; k++)
+                qrow[k] = oracle_e4m3_encode((float)bf16_widen(Be[k * N + n]) / sc);
+        }
+    }
+}
+
+/*
+ * Grouped GEMM on quantised operands, dequantised exactly in fp64:
+ *   C[s, n] = a_scale[s] * b_scale[e, n] * sum_k decode(Aq[s, k]) * decode(BqT[e, n, k])
+ * for the rows s of expert e (Aq [R, K] row-major; BqT [E, N, K], K contiguous).
+ */
+void oracle_grouped_gemm_e4m3(const uint8_t *Aq, const float *a_scale, const uint8_t *BqT,
+                              const float *b_scale, const int32_t *offsets, int32_t E,
+                              int64_t K, int64_t N, double *C)
+{
+    double lut[256];
+    for (int c = 0; c < 256; c++)
+        lut[c] = oracle_e4m3_decode((uint8_t)c);
+    for (int32_t e = 0; e < E; e++) {
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t s = offsets[e]; s < offsets[e + 1]; s++) {
+            const uint8_t *a = Aq + s * K;
+            for (int64_t n = 0; n < N; n++) {
+                const uint8_t *b = BqT + ((int64_t)e * N + n) * K;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; k++)
+                    acc += lut[a[k]] * lut[b[k]];
+                C[s * N + n] = (double)a_scale[s] * (double)b_scale[(int64_t)e * N + n] * acc;
+            }
+        }
+    }
+}
+
+/* Round an fp64 value to the nearest bf16 (ties to even) and return its bits. */
+static uint16_t bf16_round(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    /* bf16 keeps 8 significant bits; scale to an integer grid of that spacing */
+    if (v == 0.0)
+        return signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    int ex;
+    frexp(a, &ex); /* a in [2^(ex-1), 2^ex) */
+    int e = ex - 1;
+    if (e < -126)
+        e = -126; /* subnormal spacing 2^-133 */
+    double step = ldexp(1.0, e - 7);
+    double q = a / step;
+    double fl = floor(q), rem = q - fl, n = fl;
+    if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0))
+        n = fl + 1.0;
+    float r = (float)(n * step); /* exact: n*step has at most 8 significant bits */
+    if (v < 0)
+        r = -r;
+    uint32_t u;
+    memcpy(&u, &r, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * The layer with its down projection in FP8 (E4M3), stage by stage:
+ *   plan -> dispatch -> GEMM1 + SwiGLU (fp64) -> h rounded to bf16 ->
+ *   h quantised per row -> GEMM2 on the quantised h and the per-column quantised
+ *   W2 (dequantised exactly) -> weighted combine (k ascending).
+ * out fp64 [M, H].  Returns an ORACLE_* status.
+ */
+int oracle_moe_ffn_fp8(const uint16_t *x, const uint16_t *W1, const uint16_t *W2,
+                       const int32_t *ids, const float *w, int64_t M, int64_t H, int64_t F,
+                       int32_t E, int32_t topk, double *out)
+{
+    int64_t R = M * (int64_t)topk;
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *perm = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    uint16_t *xp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(R ? R * H : 1));
+    uint16_t *hb = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(R ? R * F : 1));
+    uint8_t *hq = (uint8_t *)malloc((size_t)(R ? R * F : 1));
+    float *hs = (float *)malloc(sizeof(float) * (size_t)(R ? R : 1));
+    uint8_t *wq = (uint8_t *)malloc((size_t)(E * H * F));
+    float *ws = (float *)malloc(sizeof(float) * (size_t)(E * H));
+    double *yp = (double *)malloc(sizeof(double) * (size_t)(R ? R * H : 1));
+    int st = ORACLE_ERR_ARG;
+    if (!counts || !offsets || !perm || !inv || !xp || !hb || !hq || !hs || !wq || !ws || !yp)
+        goto done;
+    st = oracle_plan(ids, w, M, E, topk, counts, offsets, perm, inv, NULL);
+    if (st != ORACLE_OK)
+        goto done;
+    oracle_dispatch(x, perm, M, H, topk, xp);
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *W1e = W1 + (int64_t)e * H * 2 * F;
+#pragma omp parallel
+        {
+            double *g = (double *)malloc(sizeof(double) * (size_t)(2 * F));
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t s = offsets[e]; s < offsets[e + 1]; s++) {
+                for (int64_t j = 0; j < 2 * F; j++)
+                    g[j] = 0.0;
+                for (int64_t h = 0; h < H; h++) {
+                    double xv = bf16_widen(xp[s * H + h]);
+                    const uint16_t *wrow = W1e + h * 2 * F;
+                    for (int64_t j = 0; j < 2 * F; j++)
+                        g[j] += xv * bf16_widen(wrow[j]);
+                }
+                for (int64_t j = 0; j < F; j++)
+                    hb[s * F + j] = bf16_round(silu(g[j]) * g[F + j]);
+            }
+            free(g);
+        }
+    }
+    oracle_quantize_rows_e4m3(hb, R, F, hq, hs);
+    oracle_quantize_cols_e4m3(W2, E, F, H, wq, ws);
+    oracle_grouped_gemm_e4m3(hq, hs, wq, ws, offsets, E, F, H, yp);
+    oracle_combine(yp, inv, w, M, H, topk, out);
+done:
+    free(counts);
+    free(offsets);
+    free(perm);
+    free(inv);
+    free(xp);
+    free(hb);
+    free(hq);
+    free(hs);
+    free(wq);
+    free(ws);
+    free(yp);
+    return st;
+}
+
 int oracle_num_threads(void)
 {
     int n = 1;

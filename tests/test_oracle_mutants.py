@@ -38,6 +38,14 @@ MUTANTS = {
                                    "w[t * topk + k] = exp((double)l[out[k]]) / sum;"),
     "tile_short_edge": ("tile_row1[n] = (r + BM < offsets[e + 1]) ? r + BM : offsets[e + 1];",
                         "tile_row1[n] = r + BM;"),
+    "e4m3_ties_round_up": ("if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) != 0.0))\n        n = fl + 1.0;\n    double r",
+                           "if (rem >= 0.5)\n        n = fl + 1.0;\n    double r"),
+    "fp8_row_scale_240": ("float sc = amax > 0.0f ? amax / 448.0f : 1.0f;\n        scale[r] = sc;",
+                          "float sc = amax > 0.0f ? amax / 240.0f : 1.0f;\n        scale[r] = sc;"),
+    "fp8_cols_not_transposed": ("qrow[k] = oracle_e4m3_encode((float)bf16_widen(Be[k * N + n]) / sc);",
+                                "qrow[k] = oracle_e4m3_encode((float)bf16_widen(Be[n * K + k]) / sc);"),
+    "fp8_gemm_drops_b_scale": ("C[s * N + n] = (double)a_scale[s] * (double)b_scale[(int64_t)e * N + n] * acc;",
+                               "C[s * N + n] = (double)a_scale[s] * acc;"),
 }
 
 CHILD = textwrap.dedent("""
@@ -46,7 +54,16 @@ CHILD = textwrap.dedent("""
     import oracle
     oracle._lib = oracle.configure(ctypes.CDLL({lib!r}))
     import test_oracle_pins as pins
+    import test_oracle_fp8_pins as fp8
     calls = [
+        fp8.test_decode_every_code_matches_torch,
+        fp8.test_encode_matches_torch_and_brute_force,
+        fp8.test_encode_saturates,
+        fp8.test_quantize_rows_matches_torch_and_bounds,
+        fp8.test_quantize_cols_matches_torch,
+        fp8.test_grouped_gemm_e4m3_matches_numpy,
+        fp8.test_fp8_layer_dense_special_case,
+        lambda: fp8.test_fp8_layer_within_e4m3_bound_of_exact_layer(64, 4, 2),
         lambda: pins.test_plan_matches_stable_sort(33, 8, 2, True),
         lambda: pins.test_plan_matches_stable_sort(50, 5, 3, False),
         pins.test_tiling_worked_example,
