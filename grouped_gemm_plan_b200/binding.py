@@ -24,13 +24,15 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
                 8: "MOE_ERR_BAD_INDEX"}
 
 EPI_STORE, EPI_SWIGLU, EPI_WEIGHT_SCATTER = 0, 1, 2
-OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE = 0, 1, 2, 3, 4, 5
+OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FFN_FP8 = \
+    0, 1, 2, 3, 4, 5, 6
 
 # Every symbol include/moe.h declares.
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_plan", "moe_dispatch",
            "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
-           "moe_set_stage_events", "moe_last_error"]
+           "moe_set_stage_events", "moe_quantize_weights_e4m3", "moe_quantize_rows_e4m3",
+           "moe_grouped_gemm_e4m3", "moe_ffn_fused_fp8", "moe_last_error"]
 
 
 class MoEError(RuntimeError):
@@ -81,6 +83,15 @@ def load(path: str | None = None):
     lib.moe_set_wait_timeout_ns.restype = None
     lib.moe_set_fault_injection.argtypes = [i32, i32]
     lib.moe_set_fault_injection.restype = st
+    lib.moe_quantize_weights_e4m3.argtypes = [P, i32, i64, i64, P, P, P]
+    lib.moe_quantize_weights_e4m3.restype = st
+    lib.moe_quantize_rows_e4m3.argtypes = [P, i64, i64, P, P, P, sz, P]
+    lib.moe_quantize_rows_e4m3.restype = st
+    lib.moe_grouped_gemm_e4m3.argtypes = [P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, sz, P]
+    lib.moe_grouped_gemm_e4m3.restype = st
+    lib.moe_ffn_fused_fp8.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P, sz,
+                                      P]
+    lib.moe_ffn_fused_fp8.restype = st
     lib.moe_set_stage_events.argtypes = [P]
     lib.moe_set_stage_events.restype = st
     lib.moe_last_error.restype = ctypes.c_char_p
@@ -183,6 +194,44 @@ def moe_ffn_fused_noalloc(x, W1, W2, topk_ids, topk_w, out, counts, offsets, per
     _check(load().moe_ffn_fused_noalloc(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w),
                                         M, H, F2 // 2, E, topk, _ptr(out), _ptr(counts),
                                         _ptr(offsets), _ptr(perm), _ptr(status), _stream(stream)))
+
+
+def moe_quantize_weights_e4m3(W, Wq, scale, stream=None):
+    """W bf16 [E, K, N] -> Wq uint8 [E, N, K] (E4M3 codes, K contiguous), scale fp32 [E, N]."""
+    E, K, N = W.shape
+    _check(load().moe_quantize_weights_e4m3(_ptr(W), E, K, N, _ptr(Wq), _ptr(scale),
+                                            _stream(stream)))
+
+
+def moe_quantize_rows_e4m3(A, Aq, scale, ws, stream=None):
+    """A bf16 [R, K] -> Aq uint8 [R, K] (E4M3 codes), scale fp32 [R]."""
+    R, K = A.shape
+    _check(load().moe_quantize_rows_e4m3(_ptr(A), R, K, _ptr(Aq), _ptr(scale), _ptr(ws),
+                                         ws.numel(), _stream(stream)))
+
+
+def moe_grouped_gemm_e4m3(Aq, a_scale, BqT, b_scale, offsets, C, ws, w_sorted=None, perm=None,
+                          stream=None):
+    """C fp32 [R, N] from E4M3 Aq [R, K] and BqT [E, N, K] (see include/moe.h)."""
+    R, K = Aq.shape
+    E, N, K2 = BqT.shape
+    if K2 != K:
+        raise ValueError(f"Aq has K={K} but BqT has K={K2}")
+    _check(load().moe_grouped_gemm_e4m3(_ptr(Aq), _ptr(a_scale), _ptr(BqT), _ptr(b_scale),
+                                        _ptr(offsets), E, R, K, N, _ptr(w_sorted), _ptr(perm),
+                                        _ptr(C), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_ffn_fused_fp8(x, W1, W2q, w2_scale, topk_ids, topk_w, out, counts, offsets, perm, ws,
+                      stream=None):
+    """The layer with the E4M3 down projection; W2q / w2_scale from moe_quantize_weights_e4m3."""
+    M, H = x.shape
+    E, _, F2 = W1.shape
+    topk = topk_ids.shape[1]
+    _check(load().moe_ffn_fused_fp8(_ptr(x), _ptr(W1), _ptr(W2q), _ptr(w2_scale), _ptr(topk_ids),
+                                    _ptr(topk_w), M, H, F2 // 2, E, topk, _ptr(out), _ptr(counts),
+                                    _ptr(offsets), _ptr(perm), _ptr(ws), ws.numel(),
+                                    _stream(stream)))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

@@ -25,6 +25,15 @@ int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, in
                         const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                         int num_sms, cudaStream_t stream);
 size_t layer_sync_bytes(int64_t M, int64_t R, int32_t E);
+cudaError_t launch_quantize_rows(const void* A, int64_t R, int64_t K, void* q, float* scale,
+                                 int num_sms, cudaStream_t stream);
+cudaError_t launch_quantize_cols(const void* W, int32_t E, int64_t K, int64_t N, void* qT,
+                                 float* scale, cudaStream_t stream);
+int launch_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* BqT,
+                             const float* b_scale, const int32_t* offsets, int32_t E, int64_t R,
+                             int64_t K, int64_t N, const float* w_sorted, const int32_t* perm,
+                             float* C, int32_t* status, uint64_t timeout_ns, int num_sms,
+                             cudaStream_t stream);
 int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_t* perm,
                      const float* w_sorted, const int32_t* offsets, void* xp, void* h, void* yk,
                      void* out, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk,
@@ -116,6 +125,25 @@ FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t top
   return L;
 }
 
+// moe_ffn_fused_fp8: the bf16 layout, then the quantised h and its row scales.
+struct Fp8Layout {
+  FusedLayout base;
+  size_t hq, hs, total;
+};
+
+Fp8Layout fp8_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
+  const int64_t R = M * topk;
+  Fp8Layout L;
+  L.base = fused_layout(M, H, F, E, topk);
+  size_t off = L.base.total;
+  L.hq = off;
+  off += align256(size_t(R) * size_t(F));
+  L.hs = off;
+  off += align256(size_t(R) * 4);
+  L.total = off;
+  return L;
+}
+
 moe_status check_ws(moe_op op, void* ws, size_t ws_bytes, int64_t M, int64_t H, int64_t F,
                     int32_t E, int32_t topk) {
   if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
@@ -183,6 +211,7 @@ moe_status moe_set_fault_injection(int32_t kind, int32_t index) {
 size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
   if (M < 0 || H < 0 || F < 0 || topk < 0 || E < 1 || E > MOE_MAX_EXPERTS) return kCtrlBytes;
   if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, E, topk).total;
+  if (op == MOE_OP_FFN_FP8) return fp8_layout(M, H, F, E, topk).total;
   if (op == MOE_OP_PLAN) return kCtrlBytes + plan_scratch_bytes(E);
   return kCtrlBytes;
 }
@@ -383,6 +412,125 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
   err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused combine");
   stage_mark(5, s);
+  return MOE_OK;
+}
+
+moe_status moe_quantize_weights_e4m3(const void* W, int32_t E, int64_t K, int64_t N, void* Wq,
+                                     float* scale, void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (K <= 0 || K % 16 != 0 || N <= 0 || N % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld and N = %lld must be positive multiples of 16", (long long)K, (long long)N);
+  if (K > kMaxRows || N > kMaxRows || int64_t(E) * N > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N too large");
+  if (W == nullptr || Wq == nullptr || scale == nullptr) return fail(MOE_ERR_INVALID_ARG, "W, Wq and scale must not be NULL");
+  if (!aligned16(W) || !aligned16(Wq)) return fail(MOE_ERR_MISALIGNED, "W and Wq must be 16-byte aligned");
+  const cudaError_t err = moe::launch_quantize_cols(W, E, K, N, Wq, scale, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_weights_e4m3");
+}
+
+moe_status moe_quantize_rows_e4m3(const void* A, int64_t R, int64_t K, void* Aq, float* scale,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 64 != 0 || K > 32768)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64, at most 32768", (long long)K);
+  moe_status st = check_ws(MOE_OP_GROUPED_GEMM, ws, ws_bytes, R, K, K, 1, 1);
+  if (st != MOE_OK) return st;
+  if (R == 0) return MOE_OK;
+  if (A == nullptr || Aq == nullptr || scale == nullptr) return fail(MOE_ERR_INVALID_ARG, "A, Aq and scale must not be NULL");
+  if (!aligned16(A) || !aligned16(Aq)) return fail(MOE_ERR_MISALIGNED, "A and Aq must be 16-byte aligned");
+  const cudaError_t err = moe::launch_quantize_rows(A, R, K, Aq, scale, num_sms_current(),
+                                                    reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_rows_e4m3");
+}
+
+moe_status moe_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* BqT,
+                                 const float* b_scale, const int32_t* offsets, int32_t E,
+                                 int64_t R, int64_t K, int64_t N, const float* w_sorted,
+                                 const int32_t* perm, float* C, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64", (long long)K);
+  if (N <= 0 || N % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "N = %lld must be a positive multiple of 64", (long long)N);
+  if (K > (int64_t(1) << 30) || N > (int64_t(1) << 30) || int64_t(E) * N > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N too large");
+  moe_status st = check_ws(MOE_OP_GROUPED_GEMM, ws, ws_bytes, R, N, K, E, 1);
+  if (st != MOE_OK) return st;
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets must not be NULL");
+  if (R == 0) return MOE_OK;
+  if (Aq == nullptr || BqT == nullptr || C == nullptr || a_scale == nullptr || b_scale == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "Aq, a_scale, BqT, b_scale and C must not be NULL");
+  if (!aligned16(Aq) || !aligned16(BqT) || !aligned16(C))
+    return fail(MOE_ERR_MISALIGNED, "Aq, BqT and C must be 16-byte aligned");
+  const int rc = moe::launch_grouped_gemm_e4m3(Aq, a_scale, BqT, b_scale, offsets, E, R, K, N,
+                                               w_sorted, perm, C, status_word(ws), g_timeout_ns,
+                                               num_sms_current(),
+                                               reinterpret_cast<cudaStream_t>(stream));
+  if (rc == 1) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_grouped_gemm_e4m3 launch");
+  return MOE_OK;
+}
+
+moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
+                             const float* w2_scale, const int32_t* topk_ids, const float* topk_w,
+                             int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk, void* out,
+                             int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
+                             size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  if (H <= 0 || H % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 64", (long long)H);
+  if (F <= 0 || F % 64 != 0 || F > 32768) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be a positive multiple of 64, at most 32768", (long long)F);
+  if (H > (int64_t(1) << 30) || int64_t(E) * H > kMaxRows || int64_t(E) * F > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
+  st = check_ws(MOE_OP_FFN_FP8, ws, ws_bytes, M, H, F, E, topk);
+  if (st != MOE_OK) return st;
+  if (counts == nullptr || offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current();
+  if (M == 0) {
+    cudaError_t err = moe::launch_plan(topk_ids, topk_w, 0, E, counts, offsets, perm, nullptr,
+                                       nullptr, status_word(ws), plan_scratch(ws), sms, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ffn_fused_fp8 plan");
+  }
+  if (x == nullptr || W1 == nullptr || W2q == nullptr || w2_scale == nullptr || topk_ids == nullptr ||
+      topk_w == nullptr || out == nullptr || perm == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "x, W1, W2q, w2_scale, topk_ids, topk_w, out and perm must not be NULL");
+  if (!aligned16(x) || !aligned16(W1) || !aligned16(W2q) || !aligned16(out))
+    return fail(MOE_ERR_MISALIGNED, "x, W1, W2q and out must be 16-byte aligned");
+  const int64_t R = M * topk;
+  moe::PdlScope pdl(static_cast<double>(R) * static_cast<double>(H) * static_cast<double>(F) <
+                    4294967296.0);
+  const Fp8Layout L = fp8_layout(M, H, F, E, topk);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* xp = base + L.base.xp;
+  void* h = base + L.base.h;
+  float* yk = reinterpret_cast<float*>(base + L.base.yk);
+  float* w_sorted = reinterpret_cast<float*>(base + L.base.w_sorted);
+  void* hq = base + L.hq;
+  float* hs = reinterpret_cast<float*>(base + L.hs);
+  int32_t* status = status_word(ws);
+
+  cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
+                                     perm, nullptr, w_sorted, status, plan_scratch(ws), sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 plan");
+  err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 dispatch");
+  int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,
+                                    nullptr, h, status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM1)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused_fp8 GEMM1");
+  err = moe::launch_quantize_rows(h, R, F, hq, hs, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 quantise");
+  rc = moe::launch_grouped_gemm_e4m3(hq, hs, W2q, w2_scale, offsets, E, R, F, H, w_sorted, perm,
+                                     yk, status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (FP8 GEMM2)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused_fp8 GEMM2");
+  err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 combine");
   return MOE_OK;
 }
 

@@ -87,7 +87,8 @@ typedef enum moe_op {
   MOE_OP_GROUPED_GEMM = 2,
   MOE_OP_COMBINE = 3,
   MOE_OP_FFN_FUSED = 4,
-  MOE_OP_ROUTE = 5
+  MOE_OP_ROUTE = 5,
+  MOE_OP_FFN_FP8 = 6   /* moe_ffn_fused_fp8 */
 } moe_op;
 
 /* Version of this ABI (incremented on any incompatible change). */
@@ -243,6 +244,58 @@ moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const void* W2,
                                  int64_t H, int64_t F, int32_t E, int32_t topk, void* out,
                                  int32_t* counts, int32_t* offsets, int32_t* perm,
                                  int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------- FP8 (E4M3)
+ * The down projection on 8-bit floats ([PTO] "MegaMoE 融合算子七阶段": SwiGLU
+ * consumes each GMM1 segment and quantises it, so that GMM2 runs on quantised
+ * activations).  E4M3 is the 8-bit float with 4 exponent bits (bias 7), 3
+ * mantissa bits, no infinities, largest finite 448.  A quantised value is
+ * q = nearest E4M3 to (v / scale) computed in fp32, ties to even, saturating at
+ * 448; scale = (largest |v| of its group) / 448 in fp32, 1 for an all-zero
+ * group, so that v ~= scale * q and the group's largest element maps to +-448.
+ */
+
+/* moe_quantize_weights_e4m3 -- offline, once per weight tensor:
+ *   W bf16 [E, K, N] row-major (the layout of W2, N contiguous)
+ *   Wq  E4M3 bytes [E, N, K] (K contiguous: the K-major operand of the FP8 GEMM)
+ *   scale fp32 [E, N]: one scale per (expert, output column), over K.
+ * K and N must be multiples of 16.  All pointers device, caller-owned. */
+moe_status moe_quantize_weights_e4m3(const void* W, int32_t E, int64_t K, int64_t N, void* Wq,
+                                     float* scale, void* stream);
+
+/* moe_quantize_rows_e4m3 -- per-row quantisation of a bf16 matrix:
+ *   A bf16 [R, K] -> Aq E4M3 bytes [R, K], scale fp32 [R] (one per row).
+ * K must be a multiple of 64 and at most 32768.  Workspace as for
+ * MOE_OP_GROUPED_GEMM (the status word). */
+moe_status moe_quantize_rows_e4m3(const void* A, int64_t R, int64_t K, void* Aq, float* scale,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* moe_grouped_gemm_e4m3 -- grouped GEMM on E4M3 operands (tcgen05 kind::f8f6f4,
+ * fp32 accumulate), the FP8 counterpart of moe_grouped_gemm with the
+ * MOE_EPI_WEIGHT_SCATTER epilogue:
+ *   for every expert e and row s in [offsets[e], offsets[e+1]):
+ *     C[d, n] = w * a_scale[s] * b_scale[e, n] * sum_k Aq[s, k] * BqT[e, n, k]
+ *   with d = perm[s], w = w_sorted[s] (perm == NULL: d = s; w_sorted == NULL:
+ *   w = 1).  Aq [R, K] and BqT [E, N, K] as written by the two quantisers
+ *   (K contiguous), C fp32 [R, N].  K and N must be multiples of 64.  Workspace
+ *   as for MOE_OP_GROUPED_GEMM. */
+moe_status moe_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* BqT,
+                                 const float* b_scale, const int32_t* offsets, int32_t E,
+                                 int64_t R, int64_t K, int64_t N, const float* w_sorted,
+                                 const int32_t* perm, float* C, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* moe_ffn_fused_fp8 -- the layer with an FP8 down projection:
+ *   plan -> dispatch -> GEMM1 + SwiGLU (bf16 h, as moe_ffn_fused) -> h
+ *   quantised per row -> FP8 GEMM2 against W2q / w2_scale (from
+ *   moe_quantize_weights_e4m3 on W2 [E, F, H]) with the gate-weight scatter ->
+ *   combine.  Arguments as moe_ffn_fused (without n_c); the workspace is
+ *   moe_workspace_size(MOE_OP_FFN_FP8, ...).  F at most 32768. */
+moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
+                             const float* w2_scale, const int32_t* topk_ids, const float* topk_w,
+                             int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk, void* out,
+                             int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns the device status word of `ws` (a moe_status)
  * and clears it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error. */
