@@ -135,6 +135,39 @@ def test_fused_validation(lib):
     assert f(*args(ws=need - 1)) == 4
 
 
+def test_fp8_validation(lib):
+    qw = lib.moe_quantize_weights_e4m3
+    assert qw(FAKE, 0, 64, 64, FAKE, FAKE, None) == 2               # E
+    assert qw(FAKE, 2, 40, 64, FAKE, FAKE, None) == 2               # K % 16
+    assert qw(None, 2, 64, 64, FAKE, FAKE, None) == 1               # null W
+    assert qw(ctypes.c_void_p(0x10008), 2, 64, 64, FAKE, FAKE, None) == 7
+    qr = lib.moe_quantize_rows_e4m3
+    assert qr(FAKE, 4, 96, FAKE, FAKE, FAKE_WS, 256, None) == 2     # K % 64
+    assert qr(FAKE, 4, 32832, FAKE, FAKE, FAKE_WS, 256, None) == 2  # K > 32768
+    assert qr(FAKE, -1, 64, FAKE, FAKE, FAKE_WS, 256, None) == 1
+    assert qr(FAKE, 4, 64, FAKE, FAKE, FAKE_WS, 100, None) == 4     # workspace
+    assert qr(None, 0, 64, None, None, FAKE_WS, 256, None) == 0     # R = 0: no-op
+    g = lib.moe_grouped_gemm_e4m3
+    args = lambda **kw: [kw.get("A", FAKE), FAKE, FAKE, FAKE, FAKE, kw.get("E", 4), kw.get("R", 64),
+                         kw.get("K", 128), kw.get("N", 256), None, None, FAKE, FAKE_WS, 256, None]
+    assert g(*args(K=100)) == 2
+    assert g(*args(N=96)) == 2
+    assert g(*args(E=0)) == 2
+    assert g(*args(R=-1)) == 1
+    assert g(*args(A=None)) == 1
+    assert g(*args(A=ctypes.c_void_p(0x10008))) == 7
+    f = lib.moe_ffn_fused_fp8
+    need = B.moe_workspace_size(B.OP_FFN_FP8, 16, 128, 128, 4, 2)
+    assert need >= B.moe_workspace_size(B.OP_FFN_FUSED, 16, 128, 128, 4, 2) + 32 * 128
+    fa = lambda **kw: [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("M", 16), kw.get("H", 128),
+                       kw.get("F", 128), kw.get("E", 4), kw.get("topk", 2), FAKE, FAKE, FAKE, FAKE,
+                       FAKE_WS, kw.get("ws", need), None]
+    assert f(*fa(H=100)) == 2
+    assert f(*fa(F=32832)) == 2
+    assert f(*fa(topk=5)) == 1
+    assert f(*fa(ws=need - 1)) == 4
+
+
 def test_binding_rejects_cpu_tensors(lib):
     import torch
     x = torch.zeros(4, 64, dtype=torch.bfloat16)

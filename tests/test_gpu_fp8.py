@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from grouped_gemm_plan_b200 import binding as B
-from helpers import check_close, layer_case
+from helpers import check_close, guarded_empty, layer_case
 
 pytestmark = pytest.mark.gpu
 
@@ -22,9 +22,12 @@ def test_quantize_weights_matches_oracle(cuda_dev, E, K, N):
     g = torch.Generator().manual_seed(E * K + N)
     W = (torch.randn(E, K, N, generator=g) * torch.rand(1, 1, N, generator=g) / 8).to(torch.bfloat16)
     W[0, :, 1] = 0                                               # an all-zero column
-    Wq = torch.empty(E, N, K, dtype=torch.uint8, device=cuda_dev)
-    sc = torch.empty(E, N, dtype=torch.float32, device=cuda_dev)
+    Wq, check_q = guarded_empty((E, N, K), torch.uint8, cuda_dev)
+    sc, check_s = guarded_empty((E, N), torch.float32, cuda_dev)
     B.moe_quantize_weights_e4m3(W.to(cuda_dev), Wq, sc)
+    torch.cuda.synchronize()
+    check_q()
+    check_s()
     rq, rsc = oracle.quantize_cols_e4m3(W)
     assert np.array_equal(_codes(Wq), rq)
     assert np.array_equal(sc.cpu().numpy(), rsc)
@@ -35,11 +38,13 @@ def test_quantize_rows_matches_oracle(cuda_dev, R, K):
     g = torch.Generator().manual_seed(R + K)
     A = (torch.randn(R, K, generator=g) * torch.exp(torch.randn(R, 1, generator=g) * 3)).to(torch.bfloat16)
     A[R // 2] = 0
-    Aq = torch.empty(R, K, dtype=torch.uint8, device=cuda_dev)
-    sc = torch.empty(R, dtype=torch.float32, device=cuda_dev)
+    Aq, check_q = guarded_empty((R, K), torch.uint8, cuda_dev)
+    sc, check_s = guarded_empty((R,), torch.float32, cuda_dev)
     ws = B.alloc_workspace(B.OP_GROUPED_GEMM, R, K, K, 1, 1, cuda_dev)
     B.moe_quantize_rows_e4m3(A.to(cuda_dev), Aq, sc, ws)
     assert B.moe_get_device_status(ws) == B.MOE_OK
+    check_q()
+    check_s()
     rq, rsc = oracle.quantize_rows_e4m3(A)
     assert np.array_equal(_codes(Aq), rq)
     assert np.array_equal(sc.cpu().numpy(), rsc)
@@ -66,10 +71,11 @@ def test_grouped_gemm_e4m3_matches_oracle(cuda_dev, counts, K, N, scatter):
     perm = rng.permutation(R).astype(np.int32) if scatter else None
     w = rng.uniform(0.1, 1, R).astype(np.float32) if scatter else None
     d = lambda a: torch.from_numpy(a).to(cuda_dev) if a is not None else None
-    C = torch.full((R, N), float("nan"), dtype=torch.float32, device=cuda_dev)
+    C, check_c = guarded_empty((R, N), torch.float32, cuda_dev, fill=0x7F)
     ws = B.alloc_workspace(B.OP_GROUPED_GEMM, R, N, K, E, 1, cuda_dev)
     B.moe_grouped_gemm_e4m3(d(Aq), d(sa), d(Bq), d(sb), d(offsets), C, ws, w_sorted=d(w), perm=d(perm))
     assert B.moe_get_device_status(ws) == B.MOE_OK
+    check_c()
     ref = oracle.grouped_gemm_e4m3(Aq, sa, Bq, sb, offsets)
     absref = oracle.grouped_gemm_e4m3(np.where(Aq & 0x80, Aq ^ 0x80, Aq).astype(np.uint8), sa,
                                       np.where(Bq & 0x80, Bq ^ 0x80, Bq).astype(np.uint8), sb, offsets)
