@@ -16,8 +16,11 @@
 // saturating at 448 (the hardware conversion cvt.rn.satfinite via cuda_fp8.h).
 #include <cuda_fp8.h>
 
+#include <cstdlib>
+
 #include "common.cuh"
 #include "epilogue.cuh"
+#include "pair.cuh"
 
 namespace moe {
 
@@ -244,6 +247,44 @@ __device__ __forceinline__ QTile qdecode(int32_t t, const int32_t* s_tstart, con
 }
 }  // namespace
 
+// One accumulator row of a 128 x 256 (or pair-half) tile: acc * (gate weight x row
+// scale) * column scale, written in fp32 to row perm[s] (or s), columns col0 ...
+__device__ __forceinline__ void fp8_scatter_epilogue(const QArgs& args, uint32_t t_row, int32_t e,
+                                                     int32_t s, bool row_ok, int32_t col0,
+                                                     uint4* stage_buf, int lane) {
+  float rs = 0.0f;
+  float* dst = nullptr;
+  if (row_ok) {
+    int32_t dest = s;
+    float w = 1.0f;
+    if (args.perm != nullptr) dest = __ldg(args.perm + s);
+    if (args.w_sorted != nullptr) w = __ldg(args.w_sorted + s);
+    rs = w * __ldg(args.a_scale + s);
+    if (dest < 0 || dest >= args.R)
+      set_status(args.status, MOE_ERR_BAD_INDEX);
+    else
+      dst = args.C + static_cast<int64_t>(dest) * args.N + col0;
+  }
+  const float* bs = args.b_scale + static_cast<int64_t>(e) * args.N + col0;
+  const int32_t n_left = args.N - col0;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {  // 32 fp32 columns = 128 bytes per segment
+    float v[32];
+    uint4 seg[8];
+    tmem_ld32(t_row + c * 32, v);
+    tmem_ld_wait();
+    const bool in = c * 32 < n_left;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = v[i] * rs * (in ? __ldg(bs + c * 32 + i) : 0.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      seg[i] = make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                          __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+    uint8_t* d = (dst != nullptr && in) ? reinterpret_cast<uint8_t*>(dst + c * 32) : nullptr;
+    warp_store_rows128(seg, d, stage_buf, lane);
+  }
+}
+
 __global__ void __launch_bounds__(Q_THREADS, 1)
     grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const QArgs args) {
@@ -422,38 +463,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
       const uint32_t t_row = tmem_base + b * Q_BN + (static_cast<uint32_t>(q * 32) << 16);
       const bool row_ok = r < tc.rows;
       const int32_t s = tc.row0 + r;
-      const int32_t col0 = tc.ni * Q_BN;
-      float rs = 0.0f;
-      float* dst = nullptr;
-      if (row_ok) {
-        int32_t dest = s;
-        float w = 1.0f;
-        if (args.perm != nullptr) dest = __ldg(args.perm + s);
-        if (args.w_sorted != nullptr) w = __ldg(args.w_sorted + s);
-        rs = w * __ldg(args.a_scale + s);
-        if (dest < 0 || dest >= args.R)
-          set_status(args.status, MOE_ERR_BAD_INDEX);
-        else
-          dst = args.C + static_cast<int64_t>(dest) * args.N + col0;
-      }
-      const float* bs = args.b_scale + static_cast<int64_t>(tc.e) * args.N + col0;
-      const int32_t n_left = args.N - col0;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {  // 32 fp32 columns = 128 bytes per segment
-        float v[32];
-        uint4 seg[8];
-        tmem_ld32(t_row + c * 32, v);
-        tmem_ld_wait();
-        const bool in = c * 32 < n_left;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = v[i] * rs * (in ? __ldg(bs + c * 32 + i) : 0.0f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          seg[i] = make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                              __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
-        uint8_t* d = (dst != nullptr && in) ? reinterpret_cast<uint8_t*>(dst + c * 32) : nullptr;
-        warp_store_rows128(seg, d, stage_buf, lane);
-      }
+      fp8_scatter_epilogue(args, t_row, tc.e, s, row_ok, tc.ni * Q_BN, stage_buf, lane);
       tc_fence_before();
       mbar_arrive(&tempty_bar[b]);
     }
@@ -465,6 +475,261 @@ __global__ void __launch_bounds__(Q_THREADS, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, Q_TMEM_COLS);
+  }
+}
+
+
+// ---------------------------------------------------------------- FP8 GEMM on CTA pairs
+// The CTA-pair structure of grouped_gemm_2sm.cu with E4M3 operands: a cluster of
+// two CTAs shares one 256-row m-tile; each CTA loads its 128 rows of A and 128
+// rows (columns of the output) of the K-major B, the leader issues
+// tcgen05.mma.cta_group::2.kind::f8f6f4 with M = 256, N = 256, K = 32 and commits
+// to both CTAs' barriers.  A stage holds 256 of K (two 128-byte swizzle spans for
+// A and for B, 64 KB per CTA; three stages): eight MMAs per barrier round trip.
+namespace {
+constexpr int QP_BM = 256;
+constexpr int QP_BN = 256;
+constexpr int QP_BK = 256;
+constexpr int QP_STAGES = 3;
+constexpr int QP_THREADS = 192;
+constexpr int QP_BOX_BYTES = 128 * 128;             // 128 rows x 128 bytes of K
+constexpr int QP_A_BYTES = (QP_BK / 128) * QP_BOX_BYTES;
+constexpr int QP_B_BYTES = (QP_BK / 128) * QP_BOX_BYTES;
+constexpr int QP_STAGE_BYTES = QP_A_BYTES + QP_B_BYTES;
+constexpr int QP_TMEM_COLS = 512;
+constexpr int QP_DYN_SMEM = QP_STAGES * QP_STAGE_BYTES + 4 * EPI_STAGE_BYTES_PER_WARP + 1024;
+constexpr uint32_t QP_IDESC = (1u << 4) | (static_cast<uint32_t>(QP_BN >> 3) << 17) |
+                              (static_cast<uint32_t>(QP_BM >> 4) << 24);
+
+__device__ __forceinline__ QTile qdecode2(int32_t t, const int32_t* s_tstart, const int32_t* s_off,
+                                          int32_t E) {
+  int32_t lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (s_tstart[mid] <= t) lo = mid; else hi = mid;
+  }
+  const int32_t e = lo;
+  const int32_t mt = (s_off[e + 1] - s_off[e] + QP_BM - 1) / QP_BM;
+  const int32_t local = t - s_tstart[e];
+  QTile c;
+  c.e = e;
+  c.ni = local / mt;
+  const int32_t mi = local - c.ni * mt;
+  c.row0 = s_off[e] + mi * QP_BM;
+  c.rows = min(QP_BM, s_off[e + 1] - c.row0);
+  return c;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(QP_THREADS, 1)
+    grouped_gemm_e4m3_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                                 const __grid_constant__ CUtensorMap tmB, const QArgs args) {
+  extern __shared__ uint8_t qp_dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[QP_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[QP_STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int32_t s_abort;
+  __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
+  __shared__ int32_t s_tstart[MOE_MAX_EXPERTS + 1];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t E = args.E;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int32_t pair = static_cast<int32_t>(blockIdx.x) >> 1;
+  const int32_t npairs = static_cast<int32_t>(gridDim.x) >> 1;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(qp_dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  if (tid == 0) {
+    for (int s = 0; s < QP_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc2(&s_tmem_base, QP_TMEM_COLS);
+    tmem_relinquish2();
+  }
+  griddep_wait();
+  for (int e = tid; e <= E; e += QP_THREADS) s_off[e] = args.offsets[e];
+  __syncthreads();
+  if (warp == 0) {
+    int32_t bad = 0;
+    for (int e = lane; e < E; e += 32)
+      if (s_off[e] < 0 || s_off[e + 1] < s_off[e] || s_off[e + 1] > args.R) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    int32_t run = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int32_t tiles = 0;
+      if (e < E && !bad) tiles = ((s_off[e + 1] - s_off[e] + QP_BM - 1) / QP_BM) * args.n_tiles_n;
+      int32_t incl = tiles;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      if (e < E) s_tstart[e] = run + incl - tiles;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      s_tstart[E] = run;
+      if (bad && blockIdx.x == 0) set_status(args.status, MOE_ERR_BAD_INDEX);
+    }
+  }
+  // barriers of both CTAs initialised and TMEM allocated before anyone signals
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int32_t T = s_tstart[E];
+  const int32_t KB = (args.K + QP_BK - 1) / QP_BK;  // a short last k-block reads zeros
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    uint32_t stage = 0, phase = 0;
+    bool issued_any = false;
+    for (int32_t t = pair; t < T && !s_abort; t += npairs) {
+      if (t + npairs >= T) griddep_launch_dependents();
+      const QTile tc = qdecode2(t, s_tstart, s_off, E);
+      const int32_t arow = tc.row0 + 128 * static_cast<int32_t>(rank);
+      const int32_t brow = tc.ni * QP_BN + 128 * static_cast<int32_t>(rank);
+      for (int32_t kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.timeout_ns, &s_abort)) {
+          set_status(args.status, MOE_ERR_TIMEOUT);
+          s_abort = 1;
+          break;
+        }
+        const uint32_t fb = peer_addr(smem_u32(&full_bar[stage]), 0);
+        if (leader) {
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                           smem_u32(&full_bar[stage])),
+                       "r"(2 * QP_STAGE_BYTES)
+                       : "memory");
+        }
+        uint8_t* sa = ring + stage * QP_STAGE_BYTES;
+        uint8_t* sb = sa + QP_A_BYTES;
+#pragma unroll
+        for (int c = 0; c < QP_BK / 128; ++c) {
+          tma2_load_2d(sa + c * QP_BOX_BYTES, &tmA, fb, kb * QP_BK + 128 * c, arow);
+          tma2_load_3d(sb + c * QP_BOX_BYTES, &tmB, fb, kb * QP_BK + 128 * c, brow, tc.e);
+        }
+        issued_any = true;
+        if (++stage == QP_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (s_abort && issued_any) {
+      // Loads in flight complete on the leader's barrier; give them time to land.
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    uint32_t stage = 0, phase = 0, j = 0;
+    bool issued_any = false;
+    for (int32_t t = pair; t < T && !s_abort; t += npairs, ++j) {
+      const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
+      if (!mbar_wait_cluster(&tempty_bar[b], tph ^ 1u, args.timeout_ns, &s_abort)) {
+        set_status(args.status, MOE_ERR_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + b * QP_BN;
+      for (int32_t kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait_bounded(&full_bar[stage], phase, args.timeout_ns, &s_abort)) {
+          set_status(args.status, MOE_ERR_TIMEOUT);
+          s_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(ring + stage * QP_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + QP_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < QP_BK / 32; ++kk) {  // K = 32 bytes per MMA
+          const uint32_t off = (kk >> 2) * QP_BOX_BYTES + (kk & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(a_addr + off, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(b_addr + off, 16, 1024);
+          umma2_e4m3(d_tmem, adesc, bdesc, QP_IDESC, (kb | kk) != 0 ? 1u : 0u);
+        }
+        issued_any = true;
+        const uint32_t eb = smem_u32(&empty_bar[stage]);
+        umma2_commit(eb);
+        umma2_commit(peer_addr(eb, 1));
+        if (++stage == QP_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (s_abort) break;
+      const uint32_t fb = smem_u32(&tfull_bar[b]);
+      umma2_commit(fb);
+      umma2_commit(peer_addr(fb, 1));
+    }
+    if (s_abort && issued_any) {
+      umma2_commit(smem_u32(&drain_bar));
+      mbar_wait_bounded(&drain_bar, 0, args.timeout_ns, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int r = 128 * static_cast<int>(rank) + q * 32 + lane;  // row of the pair's tile
+    uint4* stage_buf = reinterpret_cast<uint4*>(ring + QP_STAGES * QP_STAGE_BYTES +
+                                                (warp - 2) * EPI_STAGE_BYTES_PER_WARP);
+    const uint32_t te_leader0 = peer_addr(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t te_leader1 = peer_addr(smem_u32(&tempty_bar[1]), 0);
+    uint32_t j = 0;
+    for (int32_t t = pair; t < T && !s_abort; t += npairs, ++j) {
+      const QTile tc = qdecode2(t, s_tstart, s_off, E);
+      const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
+      int32_t okw = 1;
+      if (lane == 0) okw = mbar_wait_bounded(&tfull_bar[b], tph, args.timeout_ns, &s_abort) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) {
+        if (lane == 0) {
+          set_status(args.status, MOE_ERR_TIMEOUT);
+          s_abort = 1;
+        }
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + b * QP_BN + (static_cast<uint32_t>(q * 32) << 16);
+      fp8_scatter_epilogue(args, t_row, tc.e, tc.row0 + r, r < tc.rows, tc.ni * QP_BN, stage_buf,
+                           lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(b == 0 ? te_leader0 : te_leader1);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer no longer touches this CTA's barriers or TMEM
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, QP_TMEM_COLS);
   }
 }
 
@@ -495,6 +760,15 @@ static bool enc_u8(CUtensorMap* m, int rank, const void* base, const cuuint64_t*
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The pair kernel when experts average at least 1024 rows (as for the bf16
+// GEMMs); MOE_GEMM_PAIR=0/1 forces one kernel.
+static bool use_pair_e4m3(int64_t R, int32_t E) {
+  const char* v = getenv("MOE_GEMM_PAIR");
+  if (v != nullptr && v[0] == '0') return false;
+  if (v != nullptr && v[0] == '1') return true;
+  return E > 0 && R >= 1024 * static_cast<int64_t>(E);
 }
 
 // C [R, N] fp32 (row perm[s] if perm is given) = w_sorted[s] * a_scale[s] *
@@ -533,9 +807,25 @@ int launch_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* B
   if (cudaGetDevice(&dev) != cudaSuccess) return 2;
   if (dev >= 31 || !(attr_mask & (1 << dev))) {
     if (cudaFuncSetAttribute(grouped_gemm_e4m3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Q_DYN_SMEM) != cudaSuccess)
+                             Q_DYN_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_e4m3_2sm_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, QP_DYN_SMEM) != cudaSuccess)
       return 2;
     if (dev < 31) attr_mask |= (1 << dev);
+  }
+  if (num_sms >= 2 && use_pair_e4m3(R, E)) {
+    // boxes of 128 rows: both CTAs of a pair load their own half of A and of B
+    CUtensorMap pA, pB;
+    const cuuint32_t pabox[2] = {128, 128};
+    const cuuint32_t pbbox[3] = {128, 128, 1};
+    if (!enc_u8(&pA, 2, Aq, adims, astr, pabox) || !enc_u8(&pB, 3, BqT, bdims, bstr, pbbox)) return 1;
+    const int64_t ptiles = (R / QP_BM + (E < R ? E : R)) * a.n_tiles_n;
+    int64_t pairs = num_sms / 2;
+    if (ptiles < pairs) pairs = ptiles;
+    if (pairs < 1) pairs = 1;
+    const cudaError_t perr = launch_pdl(grouped_gemm_e4m3_2sm_kernel, dim3(static_cast<unsigned>(2 * pairs)),
+                                        dim3(QP_THREADS), QP_DYN_SMEM, stream, 2, pA, pB, a);
+    return perr == cudaSuccess ? 0 : 2;
   }
   const int64_t tiles_max = (R / Q_BM + (E < R ? E : R)) * a.n_tiles_n;
   const int grid = static_cast<int>(tiles_max < num_sms ? tiles_max : num_sms);

@@ -56,10 +56,15 @@ def _random_codes(rng, shape):
     return c
 
 
+@pytest.mark.parametrize("pair", ["0", "1"])
 @pytest.mark.parametrize("counts,K,N,scatter", [([100, 0, 300, 29], 192, 576, True),
                                                  ([128, 256], 1408, 256, False),
-                                                 ([1, 2, 3], 128, 64, True)])
-def test_grouped_gemm_e4m3_matches_oracle(cuda_dev, counts, K, N, scatter):
+                                                 ([1, 2, 3], 128, 64, True),
+                                                 ([700, 513, 0, 256], 384, 320, True)])
+def test_grouped_gemm_e4m3_matches_oracle(cuda_dev, monkeypatch, pair, counts, K, N, scatter):
+    """Both kernels (single CTA, CTA pair): ragged experts, an empty one, K not a
+    multiple of the stage depth (zero-filled tail), a partial last column tile."""
+    monkeypatch.setenv("MOE_GEMM_PAIR", pair)
     rng = np.random.default_rng(K + N)
     E = len(counts)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
@@ -135,16 +140,19 @@ def _gpu_h(dev, x, W1, offsets, perm, topk):
     return h.cpu()
 
 
-@pytest.mark.parametrize("M,H,F,E,topk,kind", [(64, 128, 192, 4, 2, "skewed"),
-                                                (300, 256, 384, 8, 2, "uniform"),
-                                                (200, 512, 1408, 16, 4, "skewed"),
-                                                (1, 64, 128, 2, 1, "uniform")])
-def test_fp8_layer_matches_oracle(cuda_dev, M, H, F, E, topk, kind):
+@pytest.mark.parametrize("M,H,F,E,topk,kind,pair", [(64, 128, 192, 4, 2, "skewed", "0"),
+                                                     (300, 256, 384, 8, 2, "uniform", "0"),
+                                                     (200, 512, 1408, 16, 4, "skewed", "0"),
+                                                     (1, 64, 128, 2, 1, "uniform", "0"),
+                                                     (300, 256, 384, 8, 2, "uniform", "1"),
+                                                     (700, 256, 640, 2, 2, "skewed", "1")])
+def test_fp8_layer_matches_oracle(cuda_dev, monkeypatch, M, H, F, E, topk, kind, pair):
     """Element by element against the oracle's FP8 stages applied to the GPU's own
     h (the rounding of h to bf16 decides E4M3 codes, so a one-ulp difference in h
     between fp32 and fp64 accumulation can move a code by a whole E4M3 step); end
     to end against the oracle's FP8 layer from x by the relative Frobenius bar; and
     within the E4M3 error bound of the exact layer."""
+    monkeypatch.setenv("MOE_GEMM_PAIR", pair)
     w, x, W1, W2, ids, tw = layer_case(M, H, F, E, topk, kind, seed=M + F)
     W2q, w2s = _fp8_inputs(cuda_dev, W2)
     out = _run_fp8(cuda_dev, x, W1, W2q, w2s, ids, tw)
