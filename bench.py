@@ -241,7 +241,7 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------- our arm
 
-GEMM_SOURCES = ["grouped_gemm.cu", "grouped_gemm_2sm.cu", "epilogue.cuh", "common.cuh"]
+GEMM_SOURCES = ["grouped_gemm.cu", "grouped_gemm_2sm.cu", "pair.cuh", "epilogue.cuh", "common.cuh"]
 
 
 def kernel_sources_sha() -> str:
