@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(L_THREADS, 1)
       const bool two = t >= T1;
       const LTile tc = two ? decode(t - T1, a.nt2, s_ms, s_off, E) : decode(t, a.nt1, s_ms, s_off, E);
       const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
-      // one lane waits, the warp follows its verdict (keeps the warp's decision uniform)
+      // one lane waits, the warp follows its result (keeps the warp's decision uniform)
       int32_t okw = 1;
       if (lane == 0) okw = mbar_wait_layer(&tfull_bar[b], tph, sy, a.timeout_ns, &s_abort) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);

@@ -7,7 +7,7 @@ benchmark times; there the plan is compared bit for bit, a sample of output rows
 is compared with the oracle's per-token brute force, and the fused output is
 compared with the chain of separate calls over every element.
 
-Bar (the benchmark spec tolerance, read for a bf16 output): relative Frobenius <= 1e-2
+Bar (the stated layer tolerance, read for a bf16 output): relative Frobenius <= 1e-2
 and per element |err| <= 2e-2 * rms(ref) + half a bf16 ulp of ref per bf16
 rounding on the path after the last GEMM (see helpers.check_close)."""
 import numpy as np
