@@ -204,3 +204,43 @@ def test_fp8_layer_equals_chain_of_calls(cuda_dev):
     # the quantised h of the chain is the oracle's quantisation of the GPU's h
     rq, rsc = oracle.quantize_rows_e4m3(h.cpu())
     assert np.array_equal(hq.cpu().numpy(), rq) and np.array_equal(hs.cpu().numpy(), rsc)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "phi35", "qwen2"])
+def test_fp8_layer_full_size_sampled(cuda_dev, name):
+    """The FP8 layer at full size, in the launch configuration the benchmark times
+    (CTA-pair kernels on the Mixtral and Phi-3.5 shapes): the weight quantiser bit
+    for bit over all of W2, and sampled tokens against the oracle's FP8 stages on
+    the GPU's own h (E4M3 decode table, fp64 dot products)."""
+    from grouped_gemm_plan_b200 import workload as wl
+    w = wl.WORKLOADS[name]
+    dev = cuda_dev
+    x = wl.make_x(w)
+    W1 = torch.empty((w.E, w.H, 2 * w.F), dtype=torch.bfloat16, device=dev)
+    W2 = torch.empty((w.E, w.F, w.H), dtype=torch.bfloat16, device=dev)
+    wl.make_weights(w, W1, W2)
+    ids, tw = wl.make_routing(w)
+    W2q, w2s = _fp8_inputs(dev, W2)
+    rq, rs = oracle.quantize_cols_e4m3(W2.cpu())
+    assert np.array_equal(W2q.cpu().numpy(), rq) and np.array_equal(w2s.cpu().numpy(), rs)
+    out = _run_fp8(dev, x, W1, W2q, w2s, ids, tw)
+    counts, offsets, perm, inv, _ = oracle.plan(ids, tw, w.E)
+    h = _gpu_h(dev, x, W1, offsets, perm, w.topk)
+    rng = np.random.default_rng(w.seed)
+    tokens = np.unique(np.concatenate([[0, w.M - 1], rng.choice(w.M, 10, replace=False)]))
+    lut = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    pairs = [(j, int(t), k) for j, t in enumerate(tokens) for k in range(w.topk)]
+    y = {}
+    for e in sorted({int(ids[t, k]) for _, t, k in pairs}):
+        dec_w = lut[rq[e]]                                   # [H, F], decoded once per expert
+        for j, t, k in pairs:
+            if int(ids[t, k]) != e:
+                continue
+            s = int(inv[t * w.topk + k])
+            hq, hs = oracle.quantize_rows_e4m3(h[s:s + 1])
+            y[(j, k)] = (dec_w @ lut[hq[0]]) * float(hs[0]) * rs[e].astype(np.float64)
+        del dec_w
+    ref = np.zeros((len(tokens), w.H))
+    for j, t, k in pairs:                                    # k ascending, as the combine
+        ref[j] += float(tw[t, k]) * y[(j, k)]
+    check_close(out.cpu()[torch.from_numpy(tokens)], ref, f"{name} FP8 sampled rows")
