@@ -206,7 +206,7 @@ def test_fp8_layer_equals_chain_of_calls(cuda_dev):
     assert np.array_equal(hq.cpu().numpy(), rq) and np.array_equal(hs.cpu().numpy(), rsc)
 
 
-@pytest.mark.parametrize("name", ["mixtral", "phi35", "qwen2"])
+@pytest.mark.parametrize("name", ["mixtral", "phi35", "qwen2", "wide512", "wide2048"])
 def test_fp8_layer_full_size_sampled(cuda_dev, name):
     """The FP8 layer at full size, in the launch configuration the benchmark times
     (CTA-pair kernels on the Mixtral and Phi-3.5 shapes): the weight quantiser bit
