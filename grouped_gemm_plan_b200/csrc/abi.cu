@@ -17,6 +17,9 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
                         int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream);
 cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
                             void* xp, int32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_dispatch_tokens(const void* x, const int32_t* inv, int64_t M, int64_t H,
+                                   int32_t topk, void* xp, int32_t* status, int num_sms,
+                                   cudaStream_t stream);
 cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
                            int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
                            int num_sms, cudaStream_t stream);
@@ -104,7 +107,7 @@ int32_t* plan_scratch(void* ws) {
 
 // Intermediates of moe_ffn_fused inside the workspace.
 struct FusedLayout {
-  size_t xp, h, yk, w_sorted, sync, total;
+  size_t xp, h, yk, w_sorted, inv, sync, total;
 };
 
 FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
@@ -118,6 +121,8 @@ FusedLayout fused_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t top
   L.yk = off;  // fp32: the weighted rows are summed once more before the bf16 cast
   off += align256(size_t(R) * size_t(H) * 4);
   L.w_sorted = off;
+  off += align256(size_t(R) * 4);
+  L.inv = off;  // slot of every routed row (token-order dispatch)
   off += align256(size_t(R) * 4);
   L.sync = off;  // flags and counters of the single-kernel layer
   off += align256(moe::layer_sync_bytes(M, R, E));
@@ -379,8 +384,9 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   stage_mark(0, s);
+  int32_t* inv = reinterpret_cast<int32_t*>(base + L.inv);
   cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
-                                     perm, nullptr, w_sorted, status, plan_scratch(ws), sms, s);
+                                     perm, inv, w_sorted, status, plan_scratch(ws), sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused plan");
   stage_mark(1, s);
   const int32_t nc = n_c < 0 ? moe::profiled_n_c(M, H, F, E, topk) : n_c;
@@ -396,7 +402,7 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     for (int i = 2; i <= 5; ++i) stage_mark(i, s);
     return MOE_OK;
   }
-  err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
+  err = moe::launch_dispatch_tokens(x, inv, M, H, topk, xp, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused dispatch");
   stage_mark(2, s);
   int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,
@@ -514,10 +520,11 @@ moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
   float* hs = reinterpret_cast<float*>(base + L.hs);
   int32_t* status = status_word(ws);
 
+  int32_t* inv = reinterpret_cast<int32_t*>(base + L.base.inv);
   cudaError_t err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets,
-                                     perm, nullptr, w_sorted, status, plan_scratch(ws), sms, s);
+                                     perm, inv, w_sorted, status, plan_scratch(ws), sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 plan");
-  err = moe::launch_dispatch(x, perm, M, H, topk, xp, status, sms, s);
+  err = moe::launch_dispatch_tokens(x, inv, M, H, topk, xp, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 dispatch");
   int rc = moe::launch_grouped_gemm(xp, W1, offsets, E, R, H, 2 * F, MOE_EPI_SWIGLU, nullptr,
                                     nullptr, h, status, g_timeout_ns, sms, s);

@@ -59,6 +59,44 @@ __global__ void __launch_bounds__(PM_THREADS)
   }
 }
 
+// The same copy walked in token order: work item = (token t, step group q); the
+// warp loads its vectors of x[t] once and stores them to all topk slots
+// inv[t*topk + k] of the token.  Every x row is read exactly once (in slot order
+// the topk reads of a row come at different times and a large x is partly read
+// from DRAM again); the written bytes are the same.
+__global__ void __launch_bounds__(PM_THREADS)
+    dispatch_tokens_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv, int32_t M,
+                           int32_t topk, int32_t vpr, uint4* __restrict__ xp, int32_t* status) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int32_t R = M * topk;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * PM_THREADS) >> 5;
+  const int32_t groups = (vpr + 32 * DU - 1) / (32 * DU);
+  const int64_t items = static_cast<int64_t>(M) * groups;
+  for (int64_t it = (static_cast<int64_t>(blockIdx.x) * PM_THREADS + threadIdx.x) >> 5; it < items;
+       it += nwarps) {
+    const int32_t t = static_cast<int32_t>(it / groups);
+    const int32_t c0 = static_cast<int32_t>(it - static_cast<int64_t>(t) * groups) * (32 * DU) + lane;
+    const uint4* src = x + static_cast<int64_t>(t) * vpr;
+    uint4 v[DU];
+#pragma unroll
+    for (int u = 0; u < DU; ++u)
+      if (c0 + 32 * u < vpr) v[u] = __ldg(src + c0 + 32 * u);
+    for (int32_t k = 0; k < topk; ++k) {
+      const int32_t s = __ldg(inv + static_cast<int64_t>(t) * topk + k);
+      if (s < 0 || s >= R) {
+        if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+        continue;
+      }
+      uint4* dst = xp + static_cast<int64_t>(s) * vpr;
+#pragma unroll
+      for (int u = 0; u < DU; ++u)
+        if (c0 + 32 * u < vpr) dst[c0 + 32 * u] = v[u];
+    }
+  }
+}
+
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v, float wk) {
   const float2 p0 = unpack_bf16x2(v.x), p1 = unpack_bf16x2(v.y), p2 = unpack_bf16x2(v.z),
                p3 = unpack_bf16x2(v.w);
@@ -202,6 +240,17 @@ cudaError_t launch_dispatch(const void* x, const int32_t* perm, int64_t M, int64
   return launch_pdl(dispatch_kernel, dim3(grid_for_items(R * groups, num_sms)), dim3(PM_THREADS), 0,
                     stream, 1, reinterpret_cast<const uint4*>(x), perm, static_cast<int32_t>(R), topk,
                     static_cast<int32_t>(H / 8), reinterpret_cast<uint4*>(xp), status);
+}
+
+cudaError_t launch_dispatch_tokens(const void* x, const int32_t* inv, int64_t M, int64_t H,
+                                   int32_t topk, void* xp, int32_t* status, int num_sms,
+                                   cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  const int64_t groups = (H / 8 + 32 * DU - 1) / (32 * DU);
+  return launch_pdl(dispatch_tokens_kernel, dim3(grid_for_items(M * groups, num_sms)),
+                    dim3(PM_THREADS), 0, stream, 1, reinterpret_cast<const uint4*>(x), inv,
+                    static_cast<int32_t>(M), topk, static_cast<int32_t>(H / 8),
+                    reinterpret_cast<uint4*>(xp), status);
 }
 
 template <bool F32>
