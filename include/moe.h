@@ -266,7 +266,8 @@ moe_status moe_quantize_weights_e4m3(const void* W, int32_t E, int64_t K, int64_
 /* moe_quantize_rows_e4m3 -- per-row quantisation of a bf16 matrix:
  *   A bf16 [R, K] -> Aq E4M3 bytes [R, K], scale fp32 [R] (one per row).
  * K must be a multiple of 64 and at most 32768.  Workspace as for
- * MOE_OP_GROUPED_GEMM (the status word). */
+ * MOE_OP_GROUPED_GEMM (the status word).  Rows are independent; NaN inputs
+ * encode as the E4M3 NaN code.  R = 0 is a no-op. */
 moe_status moe_quantize_rows_e4m3(const void* A, int64_t R, int64_t K, void* Aq, float* scale,
                                   void* ws, size_t ws_bytes, void* stream);
 
@@ -278,7 +279,9 @@ moe_status moe_quantize_rows_e4m3(const void* A, int64_t R, int64_t K, void* Aq,
  *   with d = perm[s], w = w_sorted[s] (perm == NULL: d = s; w_sorted == NULL:
  *   w = 1).  Aq [R, K] and BqT [E, N, K] as written by the two quantisers
  *   (K contiguous), C fp32 [R, N].  K and N must be multiples of 64.  Workspace
- *   as for MOE_OP_GROUPED_GEMM. */
+ *   as for MOE_OP_GROUPED_GEMM.  A perm entry outside [0, R) skips that row and
+ *   records MOE_ERR_BAD_INDEX; offsets inconsistent with R record it too and
+ *   compute nothing; a wait that runs out records MOE_ERR_TIMEOUT. */
 moe_status moe_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* BqT,
                                  const float* b_scale, const int32_t* offsets, int32_t E,
                                  int64_t R, int64_t K, int64_t N, const float* w_sorted,
