@@ -266,8 +266,8 @@ moe_status moe_quantize_weights_e4m3(const void* W, int32_t E, int64_t K, int64_
 /* moe_quantize_rows_e4m3 -- per-row quantisation of a bf16 matrix:
  *   A bf16 [R, K] -> Aq E4M3 bytes [R, K], scale fp32 [R] (one per row).
  * K must be a multiple of 64 and at most 32768.  Workspace as for
- * MOE_OP_GROUPED_GEMM (the status word).  Rows are independent; NaN inputs
- * encode as the E4M3 NaN code.  R = 0 is a no-op. */
+ * MOE_OP_GROUPED_GEMM (the status word).  Rows are independent.  R = 0 is a
+ * no-op. */
 moe_status moe_quantize_rows_e4m3(const void* A, int64_t R, int64_t K, void* Aq, float* scale,
                                   void* ws, size_t ws_bytes, void* stream);
 
