@@ -561,7 +561,14 @@ def run_ours(args):
               and src_clk["sm_mhz"] < 0.9 * src_clk["sm_max_mhz"])
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) if capped else pk["bf16_tflops"]
     traffic = measured_traffic("gemm1_swiglu", wl.name)
-    roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue", "bound": "tensor",
+    # which GEMM kernel the library runs for this shape (its rule: CTA pairs once
+    # experts average 1024 rows or more, unless MOE_GEMM_PAIR forces one)
+    forced = os.environ.get("MOE_GEMM_PAIR", "")
+    pair = forced == "1" or (forced != "0" and R >= 1024 * E)
+    roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue",
+                "kernel_variant": ("grouped_gemm_2sm_kernel (CTA pair, 256x256 tiles)" if pair
+                                   else "grouped_gemm_kernel (single CTA, 128x256 tiles)"),
+                "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{pk_kind} " + ("bf16_tflops_sustained (SM clock dropped under the "
                                                  "power cap)" if capped else "bf16_tflops (burst)"),
