@@ -60,7 +60,8 @@ def _random_codes(rng, shape):
 @pytest.mark.parametrize("counts,K,N,scatter", [([100, 0, 300, 29], 192, 576, True),
                                                  ([128, 256], 1408, 256, False),
                                                  ([1, 2, 3], 128, 64, True),
-                                                 ([700, 513, 0, 256], 384, 320, True)])
+                                                 ([700, 513, 0, 256], 384, 320, True),
+                                                 ([i % 4 for i in range(1024)], 128, 64, True)])
 def test_grouped_gemm_e4m3_matches_oracle(cuda_dev, monkeypatch, pair, counts, K, N, scatter):
     """Both kernels (single CTA, CTA pair): ragged experts, an empty one, K not a
     multiple of the stage depth (zero-filled tail), a partial last column tile."""

@@ -77,6 +77,7 @@ MEDIUM = [
     (1000, 128, 256, 64, 4, "skewed"),    # many small experts, most tiles ragged
     (64, 1024, 512, 16, 8, "skewed"),     # wide top-k, tiny M
     (513, 256, 128, 1, 1, "uniform"),     # dense special case E = 1, topk = 1
+    (300, 64, 64, 1024, 8, "uniform"),    # the largest expert count: most experts hold 0-5 rows
 ]
 
 
