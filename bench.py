@@ -228,7 +228,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * wl.M / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "M": wl.M, "H": wl.H, "F": wl.F, "E": wl.E,
-                   "topk": wl.topk, "routing": wl.routing, "seed": wl.seed},
+                   "topk": wl.topk, "routing": wl.routing, "std": wl.std, "seed": wl.seed},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n_tok} tokens per step of the {wl.name} batch, per-token "
                                    f"brute force in fp64"},
