@@ -168,6 +168,12 @@ def test_fp8_validation(lib):
     assert f(*fa(ws=need - 1)) == 4
 
 
+def test_stage_events_switch(lib):
+    # off is always accepted; no CUDA call is made until a layer runs
+    assert lib.moe_set_stage_events(None) == 0
+    assert lib.moe_set_stage_events(None) == 0
+
+
 def test_binding_rejects_cpu_tensors(lib):
     import torch
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
