@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
                 8: "MOE_ERR_BAD_INDEX"}
 
 EPI_STORE, EPI_SWIGLU, EPI_WEIGHT_SCATTER = 0, 1, 2
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024   # MOE_NOALLOC_SCRATCH_BYTES
 OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FFN_FP8 = \
     0, 1, 2, 3, 4, 5, 6
 

@@ -4,6 +4,7 @@
 // workspace carving, and kernel launches on the caller's stream.  Every step of
 // the layer itself runs in the kernels of plan.cu, permute.cu and
 // grouped_gemm.cu; there is no host or CPU fallback.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -83,17 +84,17 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int num_sms_current() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];  // zero-initialised (static storage)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 int32_t* status_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
@@ -167,7 +168,7 @@ moe_status check_route(int64_t M, int32_t E, int32_t topk) {
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d > %d", E, MOE_MAX_EXPERTS);
   if (topk < 1 || topk > E) return fail(MOE_ERR_INVALID_ARG, "topk = %d not in [1, E=%d]", topk, E);
   if (topk > 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "topk = %d > 32", topk);
-  if (M * topk > kMaxRows) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "M*topk exceeds 2^31-1");
+  if (M > kMaxRows / topk) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "M*topk exceeds 2^31-1");
   return MOE_OK;
 }
 
@@ -179,7 +180,21 @@ moe_status record_error(moe_status st, const std::string& msg) {
   g_last_error = msg;
   return st;
 }
+void clear_last_error() { g_last_error.clear(); }
 uint64_t wait_timeout_ns() { return g_timeout_ns; }
+
+// The shape checks of the whole layer (moe_ffn_fused and its variants): the
+// routing sizes, H and F positive multiples of 64, and every row count that the
+// kernels hold in int32 within range.  Records the message; returns the status.
+moe_status check_layer_shape(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  if (H <= 0 || H % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 64", (long long)H);
+  if (F <= 0 || F % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be a positive multiple of 64", (long long)F);
+  if (H > (int64_t(1) << 30) || F > (int64_t(1) << 29) || int64_t(E) * H > kMaxRows || int64_t(E) * F > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
+  return MOE_OK;
+}
 }  // namespace moe
 
 extern "C" {
@@ -215,6 +230,9 @@ moe_status moe_set_fault_injection(int32_t kind, int32_t index) {
 
 size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
   if (M < 0 || H < 0 || F < 0 || topk < 0 || E < 1 || E > MOE_MAX_EXPERTS) return kCtrlBytes;
+  // sizes whose byte counts could overflow are never valid: no workspace is enough
+  if ((topk > 0 && M > kMaxRows / topk) || H > (int64_t(1) << 30) || F > (int64_t(1) << 30))
+    return SIZE_MAX;
   if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, E, topk).total;
   if (op == MOE_OP_FFN_FP8) return fp8_layout(M, H, F, E, topk).total;
   if (op == MOE_OP_PLAN) return kCtrlBytes + plan_scratch_bytes(E);
@@ -273,7 +291,7 @@ moe_status moe_route(const float* logits, int64_t M, int32_t E, int32_t topk, in
 moe_status moe_dispatch(const void* x, const int32_t* perm, int64_t M, int64_t H, int32_t topk,
                         void* xp, void* ws, size_t ws_bytes, void* stream) {
   g_last_error.clear();
-  if (M < 0 || topk < 1 || topk > 32 || M * topk > kMaxRows)
+  if (M < 0 || topk < 1 || topk > 32 || M > kMaxRows / topk)
     return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
   if (H <= 0 || H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 8", (long long)H);
   moe_status st = check_ws(MOE_OP_DISPATCH, ws, ws_bytes, M, H, 0, 1, topk);
@@ -292,7 +310,7 @@ moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
                        const float* topk_w, int64_t M, int64_t H, int32_t topk, void* out,
                        void* ws, size_t ws_bytes, void* stream) {
   g_last_error.clear();
-  if (M < 0 || topk < 1 || topk > 32 || M * topk > kMaxRows)
+  if (M < 0 || topk < 1 || topk > 32 || M > kMaxRows / topk)
     return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
   if (H <= 0 || H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 8", (long long)H);
   moe_status st = check_ws(MOE_OP_COMBINE, ws, ws_bytes, M, H, 0, 1, topk);
@@ -345,12 +363,8 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
                          int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
                          void* stream) {
   g_last_error.clear();
-  moe_status st = check_route(M, E, topk);
+  moe_status st = moe::check_layer_shape(M, H, F, E, topk);
   if (st != MOE_OK) return st;
-  if (H <= 0 || H % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 64", (long long)H);
-  if (F <= 0 || F % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be a positive multiple of 64", (long long)F);
-  if (H > (int64_t(1) << 30) || F > (int64_t(1) << 29) || int64_t(E) * H > kMaxRows || int64_t(E) * F > kMaxRows)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
   if (n_c < -1) return fail(MOE_ERR_INVALID_ARG, "n_c = %d < -1", n_c);
   st = check_ws(MOE_OP_FFN_FUSED, ws, ws_bytes, M, H, F, E, topk);
   if (st != MOE_OK) return st;
@@ -486,12 +500,9 @@ moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
                              int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
                              size_t ws_bytes, void* stream) {
   g_last_error.clear();
-  moe_status st = check_route(M, E, topk);
+  moe_status st = moe::check_layer_shape(M, H, F, E, topk);
   if (st != MOE_OK) return st;
-  if (H <= 0 || H % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 64", (long long)H);
-  if (F <= 0 || F % 64 != 0 || F > 32768) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be a positive multiple of 64, at most 32768", (long long)F);
-  if (H > (int64_t(1) << 30) || int64_t(E) * H > kMaxRows || int64_t(E) * F > kMaxRows)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
+  if (F > 32768) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "F = %lld must be at most 32768", (long long)F);
   st = check_ws(MOE_OP_FFN_FP8, ws, ws_bytes, M, H, F, E, topk);
   if (st != MOE_OK) return st;
   if (counts == nullptr || offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");

@@ -6,6 +6,7 @@
 // the caller's status word and returns false, so no kernel can spin forever.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cuda.h>
@@ -157,6 +158,54 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
+
+// ---------------------------------------------------------------- host-side set-up
+
+// The driver's cuTensorMapEncodeTiled, looked up once per process (a
+// function-local static: its initialisation is thread-safe).  nullptr if the
+// driver does not provide it.
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                       const cuuint32_t*, CUtensorMapInterleave,
+                                       CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                       CUtensorMapFloatOOBfill);
+
+inline TensorMapEncodeFn tensor_map_encoder() {
+  static const TensorMapEncodeFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<TensorMapEncodeFn>(p);
+    return static_cast<TensorMapEncodeFn>(nullptr);
+  }();
+  return fn;
+}
+
+// Set-up that must run once per device (kernel attributes such as the dynamic
+// shared-memory size).  Several host threads may call run() at once: a device's
+// bit is published with an atomic OR only after its set-up succeeded, so two
+// threads racing on the first call may both run the set-up, which sets the same
+// attributes twice and is harmless.  Devices past ordinal 63 run it every call.
+class PerDeviceOnce {
+ public:
+  template <typename Fn>
+  cudaError_t run(Fn&& fn) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    const bool tracked = dev >= 0 && dev < 64;
+    const uint64_t bit = tracked ? (uint64_t(1) << dev) : 0;
+    if (tracked && (done_.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+    err = fn();
+    if (err == cudaSuccess && tracked) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return err;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
 
 // ---------------------------------------------------------------- cross-CTA flags
 

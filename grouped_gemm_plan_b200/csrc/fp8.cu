@@ -735,26 +735,9 @@ __global__ void __launch_bounds__(QP_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-using EncodeFnQ = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                               const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFnQ encode_fn_q() {
-  static EncodeFnQ fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFnQ>(p);
-  }
-  return fn;
-}
-
 static bool enc_u8(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims,
                    const cuuint64_t* strides, const cuuint32_t* box) {
-  EncodeFnQ enc = encode_fn_q();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box,
@@ -802,17 +785,16 @@ int launch_grouped_gemm_e4m3(const void* Aq, const float* a_scale, const void* B
   a.C = C;
   a.status = status;
   a.timeout_ns = timeout_ns;
-  static int attr_mask = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 2;
-  if (dev >= 31 || !(attr_mask & (1 << dev))) {
-    if (cudaFuncSetAttribute(grouped_gemm_e4m3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Q_DYN_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_e4m3_2sm_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, QP_DYN_SMEM) != cudaSuccess)
-      return 2;
-    if (dev < 31) attr_mask |= (1 << dev);
-  }
+  static PerDeviceOnce once;
+  const cudaError_t aerr = once.run([] {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_e4m3_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Q_DYN_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(grouped_gemm_e4m3_2sm_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, QP_DYN_SMEM);
+    return e;
+  });
+  if (aerr != cudaSuccess) return 2;
   if (num_sms >= 2 && use_pair_e4m3(R, E)) {
     // boxes of 128 rows: both CTAs of a pair load their own half of A and of B
     CUtensorMap pA, pB;

@@ -540,26 +540,8 @@ __global__ void __launch_bounds__(L_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-using EncodeFnL = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                               const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFnL encode_fn() {
-  static EncodeFnL fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFnL>(p);
-  }
-  return fn;
-}
-
 static bool enc2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
-  EncodeFnL enc = encode_fn();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -571,7 +553,7 @@ static bool enc2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) 
 }
 
 static bool enc3d(CUtensorMap* m, const void* base, int64_t E, int64_t K, int64_t N) {
-  EncodeFnL enc = encode_fn();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
                         static_cast<cuuint64_t>(E)};
@@ -638,15 +620,12 @@ int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_
 
   cudaError_t err = cudaMemsetAsync(sync_area, 0, layer_sync_bytes(M, R, E), stream);
   if (err != cudaSuccess) return 2;
-  static int attr_mask = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 2;
-  if (dev >= 31 || !(attr_mask & (1 << dev))) {
-    err = cudaFuncSetAttribute(moe_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               L_DYN_SMEM);
-    if (err != cudaSuccess) return 2;
-    if (dev < 31) attr_mask |= (1 << dev);
-  }
+  static PerDeviceOnce once;
+  err = once.run([] {
+    return cudaFuncSetAttribute(moe_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L_DYN_SMEM);
+  });
+  if (err != cudaSuccess) return 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
   cfg.blockDim = dim3(L_THREADS);

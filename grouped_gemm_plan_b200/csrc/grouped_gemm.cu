@@ -341,28 +341,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFn get_encode_fn() {
-  static EncodeFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  }
-  return fn;
-}
-
 // 2D bf16 map over a row-major [rows, cols] matrix, box 64 cols x box_rows rows.
 static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
                       int box_rows) {
-  EncodeFn enc = get_encode_fn();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -375,7 +357,7 @@ static bool encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t co
 
 // 3D bf16 map over row-major [E, K, N] weights, box 64 (N) x 64 (K) x 1.
 static bool encode_3d(CUtensorMap* m, const void* base, int64_t E, int64_t K, int64_t N) {
-  EncodeFn enc = get_encode_fn();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
                         static_cast<cuuint64_t>(E)};
@@ -389,15 +371,11 @@ static bool encode_3d(CUtensorMap* m, const void* base, int64_t E, int64_t K, in
 
 template <int EPI>
 static cudaError_t set_gemm_attr_once() {
-  static int done_mask = 0;  // one bit per device ordinal (< 31)
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev < 31 && (done_mask & (1 << dev))) return cudaSuccess;
-  err = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             G_DYN_SMEM);
-  if (err == cudaSuccess && dev < 31) done_mask |= (1 << dev);
-  return err;
+  static PerDeviceOnce once;
+  return once.run([] {
+    return cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, G_DYN_SMEM);
+  });
 }
 
 int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets, int32_t E,

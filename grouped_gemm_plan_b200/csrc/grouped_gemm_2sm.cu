@@ -326,27 +326,9 @@ __global__ void __launch_bounds__(P_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-using EncodeFn2 = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                               const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFn2 encode_fn2() {
-  static EncodeFn2 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn2>(p);
-  }
-  return fn;
-}
-
 static bool enc2(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims,
                  const cuuint64_t* strides, const cuuint32_t* box) {
-  EncodeFn2 enc = encode_fn2();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
@@ -357,19 +339,16 @@ static bool enc2(CUtensorMap* m, int rank, const void* base, const cuuint64_t* d
 template <int EPI>
 static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& b,
                              const Gemm2Args& args, cudaStream_t stream) {
-  static int mask = 0;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev >= 31 || !(mask & (1 << dev))) {
-    err = cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, P_DYN_SMEM);
-    if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>,
+  static PerDeviceOnce once;
+  const cudaError_t err = once.run([] {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P_DYN_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>,
                                cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-    if (err != cudaSuccess) return err;
-    if (dev < 31) mask |= (1 << dev);
-  }
+    return e;
+  });
+  if (err != cudaSuccess) return err;
   return launch_pdl(grouped_gemm_2sm_kernel<EPI>, dim3(static_cast<unsigned>(grid)), dim3(P_THREADS),
                     P_DYN_SMEM, stream, 2, a, b, args);
 }

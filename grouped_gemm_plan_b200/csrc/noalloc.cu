@@ -33,6 +33,8 @@ int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, in
                         const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                         int num_sms, cudaStream_t stream);
 moe_status record_error(moe_status st, const std::string& msg);
+void clear_last_error();
+moe_status check_layer_shape(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
 uint64_t wait_timeout_ns();
 }  // namespace moe
 
@@ -105,13 +107,11 @@ extern "C" moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const
                                             int32_t* offsets, int32_t* perm, int32_t* status,
                                             void* stream) {
   using moe::record_error;
-  if (M < 0) return record_error(MOE_ERR_INVALID_ARG, "M < 0");
-  if (E < 1 || E > MOE_MAX_EXPERTS) return record_error(MOE_ERR_UNSUPPORTED_SHAPE, "E out of [1, MOE_MAX_EXPERTS]");
-  if (topk < 1 || topk > E || topk > 32) return record_error(MOE_ERR_INVALID_ARG, "topk out of [1, min(E, 32)]");
-  if (H <= 0 || H % 64 != 0 || F <= 0 || F % 64 != 0)
-    return record_error(MOE_ERR_UNSUPPORTED_SHAPE, "H and F must be positive multiples of 64");
-  if (H > (int64_t(1) << 30) || F > (int64_t(1) << 29))
-    return record_error(MOE_ERR_UNSUPPORTED_SHAPE, "H or F too large");
+  moe::clear_last_error();
+  // The same shape checks, with the same status codes, as moe_ffn_fused; they also
+  // bound R = M * topk and every size below, so the layout arithmetic cannot wrap.
+  const moe_status shape = moe::check_layer_shape(M, H, F, E, topk);
+  if (shape != MOE_OK) return shape;
   const int64_t R = M * topk;
   const Layout L = layout(R, H, F, E);
   if (L.total > size_t(MOE_NOALLOC_SCRATCH_BYTES))
@@ -139,7 +139,11 @@ extern "C" moe_status moe_ffn_fused_noalloc(const void* x, const void* W1, const
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   // The array keeps the previous call's contents; only the status word must
-  // start at zero (every intermediate row is written before it is read).
+  // start at zero.  On success every intermediate row is written before it is
+  // read.  When the call ends with a device error (an expert id out of range:
+  // the plan then leaves every expert empty), the GEMMs write no rows and the
+  // combine reads rows left by an earlier call, so `out` is undefined whenever
+  // the status is not MOE_OK.
   err = cudaMemsetAsync(st, 0, sizeof(int32_t), s);
   if (err == cudaSuccess)
     err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets, perm,

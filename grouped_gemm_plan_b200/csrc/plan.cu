@@ -222,16 +222,12 @@ cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E
                         int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
                         int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream) {
   const size_t smem = sizeof(int32_t) * (size_t)(2 + PLAN_WARPS) * (size_t)E;
-  static int attr_done_mask = 0;  // one bit per device ordinal (< 31)
-  int dev = 0;
-  cudaError_t aerr = cudaGetDevice(&dev);
-  if (aerr != cudaSuccess) return aerr;
-  if (dev >= 31 || !(attr_done_mask & (1 << dev))) {
-    aerr = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static PerDeviceOnce once;
+  const cudaError_t aerr = once.run([] {
+    return cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(sizeof(int32_t) * (2 + PLAN_WARPS) * MOE_MAX_EXPERTS));
-    if (aerr != cudaSuccess) return aerr;
-    if (dev < 31) attr_done_mask |= (1 << dev);
-  }
+  });
+  if (aerr != cudaSuccess) return aerr;
   if (R == 0) {
     // Only counts/offsets to write: one CTA with no rows.
     return launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), smem, stream, 1, ids, w, 0, E, 32,

@@ -226,6 +226,10 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
  * run as consecutive kernels on `stream`), plus
  *   status  int32 [1] device pointer (may be NULL): receives this call's device
  *           status word (a moe_status; MOE_ERR_BAD_EXPERT_ID etc.).
+ * Host-side checks and their status codes are those of moe_ffn_fused (shape
+ * checks first, then the scratch limit, then pointers).  When the device status
+ * is not MOE_OK (e.g. an expert id out of range), `out` is undefined: it may
+ * hold values computed from an earlier call's intermediates.
  * Limit: the intermediates of R = M*topk rows need
  *   256 + 256*(E+1)*4 + R*H*2 + R*F*2 + R*H*4 + R*4 bytes (each part rounded
  *   up to 256);

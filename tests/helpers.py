@@ -20,8 +20,16 @@ def half_ulp_bf16(r: np.ndarray) -> np.ndarray:
     return out
 
 
+# Elements allowed beyond the literal per-element bar 2e-2 * rms(ref) (without
+# the half-ulp allowance), as a fraction of all elements: the allowance exists for
+# the bf16 rounding of the largest outputs, which are rare; accumulation error
+# that pushed many elements past the literal bar would show up in this count.
+MAX_BEYOND_LITERAL_FRAC = 1e-4
+
+
 def check_close(got, ref: np.ndarray, what: str = "", rel_fro: float = REL_FRO,
-                max_abs_rms: float = MAX_ABS_RMS, ulps: float = 1.0) -> dict:
+                max_abs_rms: float = MAX_ABS_RMS, ulps: float = 1.0,
+                max_beyond_literal_frac: float | None = None) -> dict:
     """The layer's bar for a bf16 output against the fp64 oracle.
 
     relative Frobenius error <= 1e-2, and per element
@@ -30,7 +38,16 @@ def check_close(got, ref: np.ndarray, what: str = "", rel_fro: float = REL_FRO,
     only be as close as the nearest bf16 value, which is up to 2^-8 |ref| away --
     more than 2e-2 * rms(ref) for the largest elements.  ulps = 2 is used when the
     reference is itself a bf16 result (two roundings).
+
+    The count of elements beyond the literal bar 2e-2 * rms(ref) is reported
+    (``beyond_literal``).  For a single bf16 rounding (ulps = 1, the layer output
+    against the oracle) it is held to MAX_BEYOND_LITERAL_FRAC of all elements, so
+    the half-ulp allowance cannot hide accumulation error spread over many
+    elements; comparisons with more roundings only report it unless
+    ``max_beyond_literal_frac`` is given.
     """
+    if max_beyond_literal_frac is None:
+        max_beyond_literal_frac = MAX_BEYOND_LITERAL_FRAC if ulps == 1.0 else float("inf")
     g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else \
         np.asarray(got, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
@@ -43,12 +60,16 @@ def check_close(got, ref: np.ndarray, what: str = "", rel_fro: float = REL_FRO,
     rel = np.linalg.norm(g - r) / nr if nr > 0 else np.linalg.norm(g - r)
     rms = float(np.sqrt(np.mean(r * r)))
     bound = max_abs_rms * rms + ulps * half_ulp_bf16(r)
+    beyond = int((diff > max_abs_rms * rms).sum())
     stats = {"rel_fro": float(rel), "max_abs": float(diff.max()), "rms": rms,
              "max_abs_over_rms": float(diff.max() / max(rms, 1e-300)),
-             "max_excess_over_bound": float((diff - bound).max())}
+             "max_excess_over_bound": float((diff - bound).max()),
+             "beyond_literal": beyond, "elements": int(r.size)}
     assert rel <= rel_fro, f"{what}: relative Frobenius error {rel:.3e} > {rel_fro} {stats}"
     assert bool(np.all(diff <= bound)), \
         f"{what}: {int((diff > bound).sum())} elements beyond 2e-2*rms + half-ulp {stats}"
+    assert beyond <= max_beyond_literal_frac * r.size, \
+        f"{what}: {beyond} of {r.size} elements beyond the literal 2e-2*rms {stats}"
     return stats
 
 
