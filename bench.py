@@ -1,7 +1,7 @@
 #!/usr/bin/env python3
 """Benchmark of the MoE SwiGLU FFN layer on B200 (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--n-c -1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload phi35] [--n-c -1]
     python bench.py --impl reference ...      # the CPU oracle on the host cores
 
 A step is one pass of the whole layer (plan -> dispatch -> GEMM1+SwiGLU -> GEMM2
@@ -12,6 +12,12 @@ before every timed step, outside the timed events.  With N GPUs every rank runs
 its own batch (its own seed): tokens are independent, so the layer shards with
 no collective on the data path (weak scaling); the only collectives are the
 barrier and the max-over-ranks of the timings.
+
+The headline workload is the largest single-GPU configuration (the Phi-3.5-MoE
+shape).  The same line ends with a compact record of every other workload
+(``workloads``: ms/step, tokens/s, end-to-end tokens/s, GEMM fractions of the
+bf16 peak, dispatch/combine GB/s, the FP8 layer), each measured the same way
+with fewer steps.
 """
 from __future__ import annotations
 
@@ -19,6 +25,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import shutil
 import signal
 import statistics
@@ -36,6 +43,12 @@ MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "MoE-layer tokens/s"
+HEADLINE = "phi35"
+SIDE_DEFAULT = "tiny,mixtral,qwen2,wide16,wide128,wide512,wide2048"
+L2_NOTE = "GPU arm: L2 flushed (256 MiB write) before every timed step"
+# columns of one per-workload record
+SIDE_COLS = ["ms", "tok_s", "e2e_tok_s", "gemm1_frac", "gemm2_frac", "disp_GBs", "comb_GBs",
+             "fp8_ms", "fp8_gemm2_frac", "pair"]
 
 
 def parse_args(argv=None):
@@ -43,11 +56,15 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--side", default=SIDE_DEFAULT,
+                    help="comma-separated workloads recorded after the headline ('none': skip)")
+    ap.add_argument("--side-steps", type=int, default=10, dest="side_steps")
+    ap.add_argument("--side-warmup", type=int, default=3, dest="side_warmup")
     ap.add_argument("--n-c", type=int, default=-1, dest="n_c")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--n-c-sweep", default=None, dest="n_c_sweep",
                     help="comma-separated n_c values: print one timing line per value "
@@ -62,6 +79,28 @@ def peaks():
         return p, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or platform.machine()
+
+
+def workload_config(wl, world: int) -> dict:
+    """The `config` object, identical in both arms for the same workload."""
+    return {"workload": wl.name, "M": wl.M, "H": wl.H, "F": wl.F, "E": wl.E, "topk": wl.topk,
+            "routing": wl.routing, "std": wl.std, "seed": wl.seed, "l2": L2_NOTE,
+            "parallelism": f"dp{world} (independent batches, no collective)"}
+
+
+def host_threads() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -181,7 +220,7 @@ class ClockSampler:
 def oracle_inputs(wl):
     from grouped_gemm_plan_b200 import workload as W
     x = W.make_x(wl)
-    W1, W2 = W.make_weights(wl)
+    W1, W2 = W.make_weights(wl, threads=host_threads())
     ids, tw = W.make_routing(wl)
     return x, W1, W2, ids, tw
 
@@ -204,33 +243,43 @@ def oracle_tokens_per_s(wl, seconds: float, inputs=None):
 
 
 def run_reference(args):
+    """The CPU oracle as it stands, timed on the host cores: each step is a bounded
+    sample of the workload's tokens (per-token brute force in fp64)."""
     from grouped_gemm_plan_b200 import workload as W
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     wl = W.WORKLOADS[args.workload]
     import oracle
     oracle.build()
-    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
     inputs = oracle_inputs(wl)
-    vals = []
+    vals, secs = [], []
     n_tok = 0
     cores = 1
     for i in range(args.warmup + args.steps):
-        v, n, dt, cores = oracle_tokens_per_s(wl, per_step if i >= args.warmup else 0.5, inputs)
+        v, n, dt, cores = oracle_tokens_per_s(wl, per_step if i >= args.warmup else 0.25, inputs)
         if i >= args.warmup:
             vals.append(v)
+            secs.append(dt)
             n_tok = n
-    value = statistics.mean(vals)
+    value = sum(n_tok for _ in vals) / sum(secs)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * wl.M / value, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M, "H": wl.H, "F": wl.F, "E": wl.E,
-                   "topk": wl.topk, "routing": wl.routing, "std": wl.std, "seed": wl.seed},
+        # measured: wall time of one sampled step (n_tok tokens)
+        "ms_per_step": 1e3 * statistics.mean(secs),
+        "tokens_per_step": n_tok,
+        # what one full batch of M tokens would take at this rate (not measured)
+        "ms_per_full_batch_extrapolated": 1e3 * wl.M / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n_tok} tokens per step of the {wl.name} batch, per-token "
+                         "cpu_model": cpu_model(),
+                         "sample": f"{n_tok} tokens per step of the {wl.name} batch "
+                                   f"(every {max(1, wl.M // max(1, n_tok))}th token), per-token "
                                    f"brute force in fp64"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -275,6 +324,343 @@ def plan_launches(R: int, num_sms: int) -> int:
     return 1 if -(-R // (16 * seg)) <= 1 else 2
 
 
+def gemm_uses_pair(R: int, E: int) -> bool:
+    """Which GEMM kernel the library runs for this shape (its rule: CTA pairs once
+    experts average 1024 rows or more, unless MOE_GEMM_PAIR forces one)."""
+    forced = os.environ.get("MOE_GEMM_PAIR", "")
+    return forced == "1" or (forced != "0" and R >= 1024 * E)
+
+
+def stage_timing_in_step(wl) -> bool:
+    """On large layers (no programmatic dependent launch between the stages) the
+    library records an event between its stages inside the timed steps."""
+    return wl.R * wl.H * wl.F >= 2 ** 32
+
+
+def _mean_ms(pairs) -> float:
+    return statistics.mean(a.elapsed_time(b) for a, b in pairs)
+
+
+class LayerRun:
+    """One workload instance on the device, inputs resident in HBM, and the timing
+    legs run on it.  Every call goes through the public API (binding -> C ABI)."""
+
+    STAGES = ["plan", "dispatch", "gemm1_swiglu", "gemm2_scatter", "combine"]
+
+    def __init__(self, wl, dev, flush, n_c):
+        import torch
+        from grouped_gemm_plan_b200 import binding as B
+        from grouped_gemm_plan_b200 import workload as W
+        self.torch, self.B = torch, B
+        self.wl, self.dev, self.flush, self.n_c = wl, dev, flush, n_c
+        M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
+        self.x_h = W.make_x(wl).pin_memory()
+        ids_np, tw_np = W.make_routing(wl)
+        self.ids_h = torch.from_numpy(ids_np).pin_memory()
+        self.tw_h = torch.from_numpy(tw_np).pin_memory()
+        self.W1 = torch.empty((E, H, 2 * F), dtype=torch.bfloat16, device=dev)
+        self.W2 = torch.empty((E, F, H), dtype=torch.bfloat16, device=dev)
+        W.make_weights(wl, self.W1, self.W2, threads=host_threads())
+        self.x = self.x_h.to(dev)
+        self.ids = self.ids_h.to(dev)
+        self.tw = self.tw_h.to(dev)
+        self.out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(R, dtype=torch.int32, device=dev)
+        self.ws = B.alloc_workspace(B.OP_FFN_FUSED, M, H, F, E, topk, dev)
+        self.stream = torch.cuda.current_stream(dev)
+
+    def events(self, n):
+        E = self.torch.cuda.Event
+        return [(E(enable_timing=True), E(enable_timing=True)) for _ in range(n)]
+
+    def step(self, x=None, ids=None, tw=None, out=None, stream=None):
+        self.B.moe_ffn_fused(self.x if x is None else x, self.W1, self.W2,
+                             self.ids if ids is None else ids, self.tw if tw is None else tw,
+                             self.out if out is None else out, self.counts, self.offsets,
+                             self.perm, self.ws, n_c=self.n_c, stream=stream)
+
+    def check_status(self, ws, what):
+        st = self.B.moe_get_device_status(ws)
+        if st != self.B.MOE_OK:
+            raise RuntimeError(f"device status {self.B.STATUS_NAMES.get(st)} {what}")
+
+    def warm(self, warmup):
+        for _ in range(warmup):
+            self.flush.fill_(1)
+            self.step()
+        self.check_status(self.ws, "after warm-up")
+
+    def timed_steps(self, steps, barrier, clocks=None):
+        """K layer steps, L2 flushed before each; device time per step by CUDA
+        events on the launching stream, plus the library's stage events on large
+        layers.  Returns (per-step ms list, per-stage mean ms or None)."""
+        torch, B = self.torch, self.B
+        ev = self.events(steps)
+        in_step = stage_timing_in_step(self.wl)
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)] \
+            if in_step else None
+        barrier()
+        t_begin = time.monotonic()
+        for i in range(steps):
+            self.flush.fill_(1)
+            if in_step:
+                B.moe_set_stage_events(tev[i])
+            ev[i][0].record(self.stream)
+            self.step()
+            ev[i][1].record(self.stream)
+        if in_step:
+            B.moe_set_stage_events(None)
+        barrier()
+        if clocks is not None:
+            clocks.mark(t_begin, time.monotonic())
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        stages = {n: statistics.mean(tev[i][j].elapsed_time(tev[i][j + 1]) for i in range(steps))
+                  for j, n in enumerate(self.STAGES)} if in_step else None
+        self.check_status(self.ws, "in the timed region")
+        return step_ms, stages
+
+    def chain_buffers(self):
+        torch, wl, dev = self.torch, self.wl, self.dev
+        if not hasattr(self, "inv"):
+            self.inv = torch.empty(wl.R, dtype=torch.int32, device=dev)
+            self.w_sorted = torch.empty(wl.R, dtype=torch.float32, device=dev)
+            self.xp = torch.empty((wl.R, wl.H), dtype=torch.bfloat16, device=dev)
+            self.hbuf = torch.empty((wl.R, wl.F), dtype=torch.bfloat16, device=dev)
+            self.yk = torch.empty((wl.R, wl.H), dtype=torch.float32, device=dev)
+            self.out_chain = torch.empty_like(self.out)
+            self.small_ws = self.B.alloc_workspace(self.B.OP_PLAN, wl.M, wl.H, wl.F, wl.E,
+                                                   wl.topk, dev)
+
+    def chain_calls(self):
+        B, wl = self.B, self.wl
+        self.chain_buffers()
+        return [
+            lambda: B.moe_plan(self.ids, self.tw, wl.E, self.counts, self.offsets, self.perm,
+                               self.inv, self.w_sorted, self.small_ws),
+            lambda: B.moe_dispatch(self.x, self.perm, wl.topk, self.xp, self.small_ws),
+            lambda: B.moe_grouped_gemm(self.xp, self.W1, self.offsets, B.EPI_SWIGLU, self.hbuf,
+                                       self.small_ws),
+            lambda: B.moe_grouped_gemm(self.hbuf, self.W2, self.offsets, B.EPI_WEIGHT_SCATTER,
+                                       self.yk, self.small_ws, w_sorted=self.w_sorted,
+                                       perm=self.perm),
+            lambda: B.moe_combine(self.yk, None, None, wl.M, wl.topk, self.out_chain,
+                                  self.small_ws),
+        ]
+
+    def stage_loop(self, steps, barrier, clocks=None):
+        """Each stage a separate public call (the same kernels as the layer call),
+        events between them; checks that the result equals the layer call's."""
+        calls = self.chain_calls()
+        E = self.torch.cuda.Event
+        sev = [[E(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+        barrier()
+        s_begin = time.monotonic()
+        for i in range(steps):
+            self.flush.fill_(1)
+            sev[i][0].record(self.stream)
+            for j, c in enumerate(calls):
+                c()
+                sev[i][j + 1].record(self.stream)
+        barrier()
+        if clocks is not None:
+            clocks.mark(s_begin, time.monotonic())
+        self.check_status(self.small_ws, "in the stage loop")
+        assert self.torch.equal(self.out_chain.view(self.torch.int16),
+                                self.out.view(self.torch.int16)), \
+            "stage-by-stage result differs from the layer call"
+        return {n: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(steps))
+                for j, n in enumerate(self.STAGES)}
+
+    def router_us(self):
+        torch, B, wl, dev = self.torch, self.B, self.wl, self.dev
+        g = torch.Generator(device=dev).manual_seed(wl.seed)
+        logits = torch.randn((wl.M, wl.E), generator=g, device=dev, dtype=torch.float32)
+        r_ids = torch.empty((wl.M, wl.topk), dtype=torch.int32, device=dev)
+        r_w = torch.empty((wl.M, wl.topk), dtype=torch.float32, device=dev)
+        r_ws = B.alloc_workspace(B.OP_ROUTE, wl.M, 0, 0, wl.E, wl.topk, dev)
+        rev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        B.moe_route(logits, wl.topk, r_ids, r_w, r_ws)
+        rev[0].record(self.stream)
+        for _ in range(10):
+            B.moe_route(logits, wl.topk, r_ids, r_w, r_ws)
+        rev[1].record(self.stream)
+        torch.cuda.synchronize()
+        self.check_status(r_ws, "after the router")
+        return rev[0].elapsed_time(rev[1]) * 100.0
+
+    def fp8_leg(self, steps, warmup):
+        """The layer with the FP8 (E4M3) down projection: W2 quantised once
+        (offline, not timed), then K layer steps timed like the bf16 ones, and the
+        FP8 GEMM2 alone on the quantised h of a stage-by-stage pass."""
+        torch, B, wl, dev = self.torch, self.B, self.wl, self.dev
+        M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
+        W2q = torch.empty((E, H, F), dtype=torch.uint8, device=dev)
+        w2s = torch.empty((E, H), dtype=torch.float32, device=dev)
+        B.moe_quantize_weights_e4m3(self.W2, W2q, w2s)
+        ws8 = B.alloc_workspace(B.OP_FFN_FP8, M, H, F, E, topk, dev)
+        out8 = torch.empty_like(self.out)
+
+        def fp8_step():
+            B.moe_ffn_fused_fp8(self.x, self.W1, W2q, w2s, self.ids, self.tw, out8, self.counts,
+                                self.offsets, self.perm, ws8)
+        for _ in range(warmup):
+            self.flush.fill_(1)
+            fp8_step()
+        ev8 = self.events(steps)
+        for i in range(steps):
+            self.flush.fill_(1)
+            ev8[i][0].record(self.stream)
+            fp8_step()
+            ev8[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        self.check_status(ws8, "in the FP8 layer")
+        fp8_ms = _mean_ms(ev8)
+        # the FP8 GEMM2 alone: h from one stage-by-stage pass, quantised per row
+        for c in self.chain_calls()[:3]:
+            c()
+        hq = torch.empty((R, F), dtype=torch.uint8, device=dev)
+        hs = torch.empty(R, dtype=torch.float32, device=dev)
+        B.moe_quantize_rows_e4m3(self.hbuf, hq, hs, self.small_ws)
+        yk8 = torch.empty((R, H), dtype=torch.float32, device=dev)
+        g8 = self.events(steps)
+        for i in range(steps):
+            self.flush.fill_(1)
+            g8[i][0].record(self.stream)
+            B.moe_grouped_gemm_e4m3(hq, hs, W2q, w2s, self.offsets, yk8, self.small_ws,
+                                    w_sorted=self.w_sorted, perm=self.perm)
+            g8[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        self.check_status(self.small_ws, "in the FP8 GEMM2")
+        g8_ms = _mean_ms(g8)
+        of, ob = out8.float(), self.out.float()
+        rel = float(torch.linalg.norm(of - ob) / torch.linalg.norm(ob))
+        del W2q, ws8, hq, yk8, out8
+        return {"ms_per_step": fp8_ms, "gemm2_e4m3_ms": g8_ms,
+                "gemm2_e4m3_tflops": 2.0 * R * H * F / (g8_ms / 1e3) / 1e12,
+                "rel_diff_vs_bf16_layer": rel}
+
+    def e2e_ms(self, steps, barrier):
+        """End to end through the public call: every step's inputs are copied in from
+        pinned host memory and its result copied back.  As in a serving loop, step
+        i+1's upload (one copy stream) and step i-1's download (another) overlap step
+        i's compute; device inputs and outputs are double-buffered.  The timed region
+        runs from before the first upload to after the last download."""
+        torch, dev = self.torch, self.dev
+        stream = self.stream
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        bufs = [{"x": torch.empty_like(self.x), "ids": torch.empty_like(self.ids),
+                 "tw": torch.empty_like(self.tw), "out": torch.empty_like(self.out)}
+                for _ in range(2)]
+        outs_h = [torch.empty(tuple(self.out.shape), dtype=torch.bfloat16).pin_memory()
+                  for _ in range(2)]
+        n = steps
+        up_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        down_done = [torch.cuda.Event() for _ in range(n)]
+        e2e_start = torch.cuda.Event(enable_timing=True)
+        e2e_end = torch.cuda.Event(enable_timing=True)
+
+        def upload(i):
+            b = bufs[i % 2]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[i - 2])      # step i-2 has consumed this buffer
+                b["x"].copy_(self.x_h, non_blocking=True)
+                b["ids"].copy_(self.ids_h, non_blocking=True)
+                b["tw"].copy_(self.tw_h, non_blocking=True)
+                up_done[i].record(up)
+
+        barrier()
+        e2e_start.record(stream)
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            b = bufs[i % 2]
+            stream.wait_event(up_done[i])
+            if i >= 2:
+                stream.wait_event(down_done[i - 2])      # this output buffer was read back
+            self.step(b["x"], b["ids"], b["tw"], b["out"], stream=stream)
+            comp_done[i].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[i])
+                outs_h[i % 2].copy_(b["out"], non_blocking=True)
+                down_done[i].record(down)
+        stream.wait_event(down_done[n - 1])
+        e2e_end.record(stream)
+        barrier()
+        ms = e2e_start.elapsed_time(e2e_end)
+        self.check_status(self.ws, "in the end-to-end run")
+        assert torch.equal(outs_h[(n - 1) % 2].view(torch.int16),
+                           self.out.cpu().view(torch.int16)), \
+            "end-to-end result differs from the device-timed result"
+        h2d = self.x_h.numel() * 2 + self.ids_h.numel() * 4 + self.tw_h.numel() * 4
+        d2h = outs_h[0].numel() * 2
+        return ms, h2d, d2h
+
+    def rates(self, stage_ms, peak, hbm_gbs):
+        """GEMM TFLOP/s and fractions, dispatch/combine GB/s from per-stage times."""
+        wl = self.wl
+        M, H, F, R = wl.M, wl.H, wl.F, wl.R
+        g1 = 4.0 * R * H * F / (stage_ms["gemm1_swiglu"] / 1e3) / 1e12
+        g2 = 2.0 * R * H * F / (stage_ms["gemm2_scatter"] / 1e3) / 1e12
+        disp_bytes = M * H * 2 + R * H * 2 + R * 4
+        comb_bytes = R * H * 4 + M * H * 2
+        disp = disp_bytes / (stage_ms["dispatch"] / 1e3) / 1e9
+        comb = comb_bytes / (stage_ms["combine"] / 1e3) / 1e9
+        return {"gemm1_tflops": g1, "gemm2_tflops": g2,
+                "gemm1_frac": g1 / peak, "gemm2_frac": g2 / peak,
+                "dispatch_gbs": disp, "combine_gbs": comb,
+                "dispatch_frac_of_hbm": disp / hbm_gbs, "combine_frac_of_hbm": comb / hbm_gbs}
+
+    def free(self):
+        for k in list(self.__dict__):
+            if k not in ("torch", "B", "wl", "dev", "flush", "n_c", "stream"):
+                delattr(self, k)
+        self.torch.cuda.synchronize()
+        self.torch.cuda.empty_cache()
+
+
+def _r(v, digits=4):
+    """Round to `digits` significant figures (compact records)."""
+    if v is None:
+        return None
+    if v == 0:
+        return 0.0
+    from math import floor, log10
+    return float(round(v, digits - 1 - int(floor(log10(abs(v))))))
+
+
+def side_record(name, args, dev, flush, world, barrier, D, pk):
+    """One compact per-workload record: the same measurement as the headline with
+    fewer steps (stage times inside the timed steps on large layers, else from a
+    stage-by-stage loop)."""
+    from grouped_gemm_plan_b200 import workload as W
+    rank, _, _ = D.env_rank()
+    wl = D.shard(W.WORKLOADS[name], rank)
+    run = LayerRun(wl, dev, flush, args.n_c)
+    run.warm(args.side_warmup)
+    step_ms, stages = run.timed_steps(args.side_steps, barrier)
+    if stages is None:
+        stages = run.stage_loop(args.side_steps, barrier)
+    e2e, _, _ = run.e2e_ms(args.side_steps, barrier)
+    fp8 = run.fp8_leg(args.side_steps, args.side_warmup)
+    total, e2e = D.max_over_ranks([sum(step_ms), e2e], dev)
+    rates = run.rates(stages, pk["bf16_tflops"], pk["hbm_gbs"])
+    rec = [_r(total / args.side_steps), _r(D.whole_job_rate(wl.M * args.side_steps, world, total / 1e3)),
+           _r(D.whole_job_rate(wl.M * args.side_steps, world, e2e / 1e3)),
+           _r(rates["gemm1_frac"], 3), _r(rates["gemm2_frac"], 3), _r(rates["dispatch_gbs"]),
+           _r(rates["combine_gbs"]), _r(fp8["ms_per_step"]),
+           _r(fp8["gemm2_e4m3_tflops"] / (2.0 * pk["bf16_tflops"]), 3),
+           1 if gemm_uses_pair(wl.R, wl.E) else 0]
+    run.free()
+    return rec
+
+
 def run_ours(args):
     import torch
     from grouped_gemm_plan_b200 import binding as B
@@ -289,257 +675,50 @@ def run_ours(args):
     D.init("nccl", timeout_s=120, device=dev)
     B.load()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-
-    wl = D.shard(W.WORKLOADS[args.workload], rank)
-    M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
-    x_h = W.make_x(wl).pin_memory()
-    ids_np, tw_np = W.make_routing(wl)
-    ids_h = torch.from_numpy(ids_np).pin_memory()
-    tw_h = torch.from_numpy(tw_np).pin_memory()
-    W1 = torch.empty((E, H, 2 * F), dtype=torch.bfloat16, device=dev)
-    W2 = torch.empty((E, F, H), dtype=torch.bfloat16, device=dev)
-    W.make_weights(wl, W1, W2)
-    x = x_h.to(dev)
-    ids = ids_h.to(dev)
-    tw = tw_h.to(dev)
-    out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(R, dtype=torch.int32, device=dev)
-    ws = B.alloc_workspace(B.OP_FFN_FUSED, M, H, F, E, topk, dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=args.n_c)
 
     def barrier():
         D.barrier(dev)
 
+    base = W.WORKLOADS[args.workload]
+    wl = D.shard(base, rank)
+    M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
+
     if args.n_c_sweep:
+        run = LayerRun(wl, dev, flush, args.n_c)
         for nc in [int(v) for v in args.n_c_sweep.split(",")]:
-            for _ in range(args.warmup):
-                flush.fill_(1)
-                B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=nc)
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            for i in range(args.steps):
-                flush.fill_(1)
-                evs[i][0].record(stream)
-                B.moe_ffn_fused(x, W1, W2, ids, tw, out, counts, offsets, perm, ws, n_c=nc)
-                evs[i][1].record(stream)
-            torch.cuda.synchronize()
-            st = B.moe_get_device_status(ws)
-            ms = [a.elapsed_time(b) for a, b in evs]
+            run.n_c = nc
+            run.warm(args.warmup)
+            step_ms, _ = run.timed_steps(args.steps, barrier)
             if rank == 0:
-                print(json.dumps({"workload": wl.name, "n_c": nc, "status": st,
-                                  "ms_per_step": statistics.mean(ms), "ms_min": min(ms),
-                                  "tokens_per_s": M / (statistics.mean(ms) / 1e3)}), flush=True)
+                print(json.dumps({"workload": wl.name, "n_c": nc,
+                                  "ms_per_step": statistics.mean(step_ms), "ms_min": min(step_ms),
+                                  "tokens_per_s": M / (statistics.mean(step_ms) / 1e3)}),
+                      flush=True)
         D.finish()
         return 0
 
+    run = LayerRun(wl, dev, flush, args.n_c)
     clocks = ClockSampler(local)
     clocks.start()
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
-    st = B.moe_get_device_status(ws)
-    if st != B.MOE_OK:
-        raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} after warm-up")
-
-    # ---- timed region: K layer steps (the public call moe_ffn_fused), L2 flushed
-    # before each, device time by CUDA events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    # On large layers (no programmatic dependent launch between the stages, see
-    # moe_ffn_fused) the library also records an event between its stages, so the
-    # dominant kernel's duration comes from these very steps.
-    in_step = R * H * F >= 2 ** 32
-    tev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)] \
-        if in_step else None
-    barrier()
-    t_begin = time.monotonic()
-    for i in range(args.steps):
-        flush.fill_(1)
-        if in_step:
-            B.moe_set_stage_events(tev[i])
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    if in_step:
-        B.moe_set_stage_events(None)
-    barrier()
-    clocks.mark(t_begin, time.monotonic())
+    run.warm(args.warmup)
+    # ---- timed region: K layer steps (the public call moe_ffn_fused)
+    step_ms, in_step_ms = run.timed_steps(args.steps, barrier, clocks)
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    stage_names = ["plan", "dispatch", "gemm1_swiglu", "gemm2_scatter", "combine"]
-    in_step_ms = {n: statistics.mean(tev[i][j].elapsed_time(tev[i][j + 1])
-                                     for i in range(args.steps))
-                  for j, n in enumerate(stage_names)} if in_step else None
     total_ms = sum(step_ms)
-    st = B.moe_get_device_status(ws)
-    if st != B.MOE_OK:
-        raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} in the timed region")
-
-    # ---- per-kernel times: K more steps, each stage a separate public call (the
-    # same kernels as the n_c = 0 path) with events between them; its own clock
-    # record decides which measured peak the dominant kernel is held to
-    inv = torch.empty(R, dtype=torch.int32, device=dev)
-    w_sorted = torch.empty(R, dtype=torch.float32, device=dev)
-    xp = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
-    hbuf = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
-    yk = torch.empty((R, H), dtype=torch.float32, device=dev)
-    out_chain = torch.empty_like(out)
-    small_ws = B.alloc_workspace(B.OP_PLAN, M, H, F, E, topk, dev)
-    names = ["plan", "dispatch", "gemm1_swiglu", "gemm2_scatter", "combine"]
-    calls = [
-        lambda: B.moe_plan(ids, tw, E, counts, offsets, perm, inv, w_sorted, small_ws),
-        lambda: B.moe_dispatch(x, perm, topk, xp, small_ws),
-        lambda: B.moe_grouped_gemm(xp, W1, offsets, B.EPI_SWIGLU, hbuf, small_ws),
-        lambda: B.moe_grouped_gemm(hbuf, W2, offsets, B.EPI_WEIGHT_SCATTER, yk, small_ws,
-                                   w_sorted=w_sorted, perm=perm),
-        lambda: B.moe_combine(yk, None, None, M, topk, out_chain, small_ws),
-    ]
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-           for _ in range(args.steps)]
+    # ---- per-kernel times: K more steps, each stage a separate public call; its
+    # own clock record decides which measured peak the dominant kernel is held to
     sclocks = ClockSampler(local)
     sclocks.start()
-    barrier()
-    s_begin = time.monotonic()
-    for i in range(args.steps):
-        flush.fill_(1)
-        sev[i][0].record(stream)
-        for j, c in enumerate(calls):
-            c()
-            sev[i][j + 1].record(stream)
-    barrier()
-    sclocks.mark(s_begin, time.monotonic())
+    stage_avg = run.stage_loop(args.steps, barrier, sclocks)
     sclk = sclocks.stop()
-    stage_avg = {n: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1])
-                                    for i in range(args.steps))
-                 for j, n in enumerate(names)}
-    assert B.moe_get_device_status(small_ws) == B.MOE_OK
-    assert torch.equal(out_chain.view(torch.int16), out.view(torch.int16)), \
-        "stage-by-stage result differs from the layer call"
-
-    # ---- the router in front of the layer (moe_route): fp32 logits [M, E] -> ids, w
-    g = torch.Generator(device=dev).manual_seed(wl.seed)
-    logits = torch.randn((M, E), generator=g, device=dev, dtype=torch.float32)
-    r_ids = torch.empty((M, topk), dtype=torch.int32, device=dev)
-    r_w = torch.empty((M, topk), dtype=torch.float32, device=dev)
-    r_ws = B.alloc_workspace(B.OP_ROUTE, M, 0, 0, E, topk, dev)
-    rev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    B.moe_route(logits, topk, r_ids, r_w, r_ws)
-    rev[0].record(stream)
-    for _ in range(10):
-        B.moe_route(logits, topk, r_ids, r_w, r_ws)
-    rev[1].record(stream)
-    torch.cuda.synchronize()
-    router_us = rev[0].elapsed_time(rev[1]) * 100.0
-    assert B.moe_get_device_status(r_ws) == B.MOE_OK
-
-    # ---- the layer with the FP8 (E4M3) down projection (moe_ffn_fused_fp8): W2
-    # quantised once (offline step, not timed), then K steps timed like the bf16
-    # ones, and the FP8 GEMM2 alone on the quantised h of the last step
-    W2q = torch.empty((E, H, F), dtype=torch.uint8, device=dev)
-    w2s = torch.empty((E, H), dtype=torch.float32, device=dev)
-    B.moe_quantize_weights_e4m3(W2, W2q, w2s)
-    ws8 = B.alloc_workspace(B.OP_FFN_FP8, M, H, F, E, topk, dev)
-    out8 = torch.empty_like(out)
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        B.moe_ffn_fused_fp8(x, W1, W2q, w2s, ids, tw, out8, counts, offsets, perm, ws8)
-    ev8 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(1)
-        ev8[i][0].record(stream)
-        B.moe_ffn_fused_fp8(x, W1, W2q, w2s, ids, tw, out8, counts, offsets, perm, ws8)
-        ev8[i][1].record(stream)
-    torch.cuda.synchronize()
-    assert B.moe_get_device_status(ws8) == B.MOE_OK
-    fp8_ms = statistics.mean(a.elapsed_time(b) for a, b in ev8)
-    hq = torch.empty((R, F), dtype=torch.uint8, device=dev)
-    hs = torch.empty(R, dtype=torch.float32, device=dev)
-    B.moe_quantize_rows_e4m3(hbuf, hq, hs, small_ws)
-    yk8 = torch.empty((R, H), dtype=torch.float32, device=dev)
-    g8 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(1)
-        g8[i][0].record(stream)
-        B.moe_grouped_gemm_e4m3(hq, hs, W2q, w2s, offsets, yk8, small_ws, w_sorted=w_sorted,
-                                perm=perm)
-        g8[i][1].record(stream)
-    torch.cuda.synchronize()
-    assert B.moe_get_device_status(small_ws) == B.MOE_OK
-    g8_ms = statistics.mean(a.elapsed_time(b) for a, b in g8)
-    of, ob = out8.float(), out.float()
-    fp8_info = {
-        "ms_per_step": fp8_ms, "tokens_per_s": D.whole_job_rate(M, 1, fp8_ms / 1e3),
-        "gemm2_e4m3_ms": g8_ms, "gemm2_e4m3_tflops": 2.0 * R * H * F / (g8_ms / 1e3) / 1e12,
-        "rel_diff_vs_bf16_layer": float(torch.linalg.norm(of - ob) / torch.linalg.norm(ob)),
-        "how": "moe_ffn_fused_fp8 (h and W2 in E4M3, per-row / per-column fp32 scales), L2 "
-               "flushed before each step; the GEMM2 rate on the quantised h of the last step",
-    }
-    del W2q, ws8, hq, yk8
-
-    # ---- end to end: every step's inputs are copied in from pinned host memory and
-    # its result copied back, through the public call.  As in a serving loop, step
-    # i+1's upload (one copy stream) and step i-1's download (another) overlap step
-    # i's compute; device inputs and outputs are double-buffered.  The timed region
-    # runs from before the first upload to after the last download.
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    bufs = [{"x": torch.empty_like(x), "ids": torch.empty_like(ids), "tw": torch.empty_like(tw),
-             "out": torch.empty_like(out)} for _ in range(2)]
-    outs_h = [torch.empty((M, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    n = args.steps
-    up_done = [torch.cuda.Event() for _ in range(n)]
-    comp_done = [torch.cuda.Event() for _ in range(n)]
-    down_done = [torch.cuda.Event() for _ in range(n)]
-    e2e_start = torch.cuda.Event(enable_timing=True)
-    e2e_end = torch.cuda.Event(enable_timing=True)
-
-    def upload(i):
-        b = bufs[i % 2]
-        with torch.cuda.stream(up):
-            if i >= 2:
-                up.wait_event(comp_done[i - 2])      # step i-2 has consumed this buffer
-            b["x"].copy_(x_h, non_blocking=True)
-            b["ids"].copy_(ids_h, non_blocking=True)
-            b["tw"].copy_(tw_h, non_blocking=True)
-            up_done[i].record(up)
-
-    barrier()
-    e2e_start.record(stream)
-    up.wait_stream(stream)
-    down.wait_stream(stream)
-    upload(0)
-    for i in range(n):
-        if i + 1 < n:
-            upload(i + 1)
-        b = bufs[i % 2]
-        stream.wait_event(up_done[i])
-        if i >= 2:
-            stream.wait_event(down_done[i - 2])      # this output buffer was read back
-        B.moe_ffn_fused(b["x"], W1, W2, b["ids"], b["tw"], b["out"], counts, offsets, perm, ws,
-                        n_c=args.n_c, stream=stream)
-        comp_done[i].record(stream)
-        with torch.cuda.stream(down):
-            down.wait_event(comp_done[i])
-            outs_h[i % 2].copy_(b["out"], non_blocking=True)
-            down_done[i].record(down)
-    stream.wait_event(down_done[n - 1])
-    e2e_end.record(stream)
-    barrier()
-    e2e_ms = e2e_start.elapsed_time(e2e_end)
-    st = B.moe_get_device_status(ws)
-    if st != B.MOE_OK:
-        raise RuntimeError(f"device status {B.STATUS_NAMES.get(st)} in the end-to-end run")
-    assert torch.equal(outs_h[(n - 1) % 2].view(torch.int16), out.cpu().view(torch.int16)), \
-        "end-to-end result differs from the device-timed result"
-    h2d = x_h.numel() * 2 + ids_h.numel() * 4 + tw_h.numel() * 4
-    d2h = outs_h[0].numel() * 2
+    router_us = run.router_us()
+    fp8_info = run.fp8_leg(args.steps, args.warmup)
+    fp8_info["how"] = ("moe_ffn_fused_fp8 (h and W2 in E4M3, per-row / per-column fp32 scales), "
+                       "L2 flushed before each step; the GEMM2 rate on the quantised h of a "
+                       "stage-by-stage pass")
+    e2e_ms, h2d, d2h = run.e2e_ms(args.steps, barrier)
+    run.free()
 
     # ---- max over ranks
     total_ms, e2e_ms = D.max_over_ranks([total_ms, e2e_ms], dev)
@@ -551,20 +730,16 @@ def run_ours(args):
     flops_g1 = 4.0 * R * H * F
     # GEMM1's launches inside the timed steps when the library recorded them there,
     # else the separate stage-by-stage loop.
-    src_ms, src_clk = (in_step_ms, clk) if in_step else (stage_avg, sclk)
-    g1_s = src_ms["gemm1_swiglu"] / 1e3
-    achieved = flops_g1 / g1_s / 1e12
+    src_ms, src_clk = (in_step_ms, clk) if in_step_ms is not None else (stage_avg, sclk)
     # Held to the burst figure of the measured cuBLAS bf16 GEMM while the SM clock
     # stays near its maximum; to the sustained (power-capped) figure once the clock
     # has dropped.
     capped = (src_clk.get("sm_mhz") is not None and src_clk.get("sm_max_mhz")
               and src_clk["sm_mhz"] < 0.9 * src_clk["sm_max_mhz"])
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) if capped else pk["bf16_tflops"]
-    traffic = measured_traffic("gemm1_swiglu", wl.name)
-    # which GEMM kernel the library runs for this shape (its rule: CTA pairs once
-    # experts average 1024 rows or more, unless MOE_GEMM_PAIR forces one)
-    forced = os.environ.get("MOE_GEMM_PAIR", "")
-    pair = forced == "1" or (forced != "0" and R >= 1024 * E)
+    rates = run.rates(src_ms, peak, pk["hbm_gbs"])
+    achieved = rates["gemm1_tflops"]
+    pair = gemm_uses_pair(R, E)
     roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue",
                 "kernel_variant": ("grouped_gemm_2sm_kernel (CTA pair, 256x256 tiles)" if pair
                                    else "grouped_gemm_kernel (single CTA, 128x256 tiles)"),
@@ -573,31 +748,15 @@ def run_ours(args):
                 "peak_source": f"{pk_kind} " + ("bf16_tflops_sustained (SM clock dropped under the "
                                                  "power cap)" if capped else "bf16_tflops (burst)"),
                 "timed_in": ("the timed layer steps (events between the library's stage "
-                             "launches)" if in_step else "the stage-by-stage loop"),
+                             "launches)" if in_step_ms is not None else "the stage-by-stage loop"),
                 "kernel_loop_clocks": src_clk,
-                "peak_sustained": pk.get("bf16_tflops_sustained"), "traffic": traffic,
+                "peak_sustained": pk.get("bf16_tflops_sustained"),
+                "traffic": measured_traffic("gemm1_swiglu", wl.name),
                 "algorithmic": f"4*R*H*F = {flops_g1:.4g} FLOP per launch"}
-    g2 = 2.0 * R * H * F / (src_ms["gemm2_scatter"] / 1e3) / 1e12
     # E4M3 peak = the measured bf16 peak x 2 (the nominal fp8 : bf16 dense ratio)
     fp8_info["gemm2_e4m3_frac_of_fp8_peak"] = fp8_info["gemm2_e4m3_tflops"] / (2.0 * peak)
     fp8_info["fp8_peak_tflops"] = 2.0 * peak
-    disp_bytes = M * H * 2 + R * H * 2 + R * 4
-    comb_bytes = R * H * 4 + M * H * 2
-    extra = {
-        "stages_ms": stage_avg,
-        "stages_in_timed_steps_ms": in_step_ms,
-        "gemm1_tflops": achieved, "gemm2_tflops": g2,
-        "grouped_gemm_frac_of_bf16_peak": {"gemm1": achieved / peak, "gemm2": g2 / peak},
-        "dispatch_gbs": disp_bytes / (src_ms["dispatch"] / 1e3) / 1e9,
-        # read + written bytes over the measured copy bandwidth (which counts both)
-        "dispatch_frac_of_hbm": disp_bytes / (src_ms["dispatch"] / 1e3) / 1e9 / pk["hbm_gbs"],
-        "combine_frac_of_hbm": comb_bytes / (src_ms["combine"] / 1e3) / 1e9 / pk["hbm_gbs"],
-        "combine_gbs": comb_bytes / (src_ms["combine"] / 1e3) / 1e9,
-        "hbm_peak_gbs": pk["hbm_gbs"],
-        "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
-        "router_us": router_us,
-        "fp8_layer": fp8_info,
-    }
+    fp8_info["tokens_per_s"] = D.whole_job_rate(M, 1, fp8_info["ms_per_step"] / 1e3)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -605,8 +764,15 @@ def run_ours(args):
         oracle.build()
         v, n, dt, cores = oracle_tokens_per_s(W.WORKLOADS[args.workload], args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"{n} tokens of the {wl.name} batch, per-token brute force in fp64, "
                          f"{dt:.1f} s"}
+
+    side_names = [] if args.side in ("", "none") else \
+        [s for s in args.side.split(",") if s and s != args.workload]
+    side = {}
+    for name in side_names:
+        side[name] = side_record(name, args, dev, flush, world, barrier, D, pk)
 
     if rank == 0:
         line = {
@@ -614,10 +780,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "M": M, "H": H, "F": F, "E": E, "topk": topk,
-                       "routing": wl.routing, "std": wl.std, "seed": W.WORKLOADS[args.workload].seed,
-                       "n_c": args.n_c, "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"dp{world} (independent batches, no collective)"},
+            "config": workload_config(base, world),
+            "n_c": args.n_c,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
                     "how": "public call moe_ffn_fused; every step uploads x, topk_ids, topk_w "
@@ -628,7 +792,25 @@ def run_ours(args):
             "roofline": roofline,
             "cpu_baseline": cpu,
             "clocks": clk,
-            **extra,
+            "stages_ms": stage_avg,
+            "stages_in_timed_steps_ms": in_step_ms,
+            "gemm1_tflops": achieved, "gemm2_tflops": rates["gemm2_tflops"],
+            "grouped_gemm_frac_of_bf16_peak": {"gemm1": rates["gemm1_frac"],
+                                               "gemm2": rates["gemm2_frac"]},
+            "dispatch_gbs": rates["dispatch_gbs"], "combine_gbs": rates["combine_gbs"],
+            # read + written bytes over the measured copy bandwidth (which counts both)
+            "dispatch_frac_of_hbm": rates["dispatch_frac_of_hbm"],
+            "combine_frac_of_hbm": rates["combine_frac_of_hbm"],
+            "hbm_peak_gbs": pk["hbm_gbs"],
+            "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
+            "router_us": router_us,
+            "fp8_layer": fp8_info,
+            # last, so that they stay in view at the end of the line: one record per
+            # other workload, columns as named (fractions of the measured burst
+            # peaks; fp8 fraction of 2x the bf16 peak; pair = CTA-pair GEMM kernel)
+            "workloads_steps": args.side_steps,
+            "workloads_cols": SIDE_COLS,
+            "workloads": side,
         }
         print(json.dumps(line), flush=True)
     D.finish()

@@ -109,17 +109,36 @@ def make_expert_w2(wl: Workload, e: int) -> torch.Tensor:
 
 
 def make_weights(wl: Workload, out_w1: torch.Tensor | None = None,
-                 out_w2: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+                 out_w2: torch.Tensor | None = None,
+                 threads: int = 1) -> tuple[torch.Tensor, torch.Tensor]:
     """Expert weights W1 bf16 [E, H, 2F] and W2 bf16 [E, F, H].
 
     ``out_w1``/``out_w2`` may be preallocated tensors (any device) that are filled
-    expert by expert, which keeps host memory to one expert at a time.
+    expert by expert.  With ``threads`` > 1 the experts' matrices are drawn by a
+    pool of host threads (numpy releases the GIL while it fills an array); every
+    matrix has its own stream, so the values do not depend on the thread count.
+    The copies into the output tensors stay on the calling thread.
     """
     W1 = out_w1 if out_w1 is not None else torch.empty((wl.E, wl.H, 2 * wl.F), dtype=torch.bfloat16)
     W2 = out_w2 if out_w2 is not None else torch.empty((wl.E, wl.F, wl.H), dtype=torch.bfloat16)
-    for e in range(wl.E):
-        W1[e].copy_(make_expert_w1(wl, e))
-        W2[e].copy_(make_expert_w2(wl, e))
+    jobs = [(make_expert_w1, W1, e) for e in range(wl.E)] + \
+           [(make_expert_w2, W2, e) for e in range(wl.E)]
+    if threads <= 1:
+        for fn, dst, e in jobs:
+            dst[e].copy_(fn(wl, e))
+        return W1, W2
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        # submitted a few at a time, so that host memory holds about `threads`
+        # matrices rather than all of them
+        pending = []
+        for fn, dst, e in jobs:
+            pending.append((dst, e, ex.submit(fn, wl, e)))
+            if len(pending) >= 2 * threads:
+                d, i, fut = pending.pop(0)
+                d[i].copy_(fut.result())
+        for d, i, fut in pending:
+            d[i].copy_(fut.result())
     return W1, W2
 
 

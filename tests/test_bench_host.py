@@ -58,5 +58,36 @@ def test_plan_launch_count():
 
 def test_default_arguments():
     a = bench.parse_args([])
-    assert (a.gpus, a.steps, a.warmup, a.impl, a.workload) == (1, 20, 5, "ours", "mixtral")
-    assert a.warmup >= 3
+    # the headline is the largest single-GPU workload; every other one gets a record
+    assert (a.gpus, a.steps, a.warmup, a.impl, a.workload) == (1, 20, 5, "ours", "phi35")
+    assert a.warmup >= 3 and a.side_warmup >= 3
+    from grouped_gemm_plan_b200 import workload as W
+    flops = {n: W.WORKLOADS[n].flops() for n in W.WORKLOADS if n != "mixtral_prof"}
+    assert max(flops, key=flops.get) == a.workload
+    assert set(a.side.split(",")) | {a.workload} == set(flops)
+
+
+def test_compact_rounding():
+    assert bench._r(1234567.0) == 1235000.0
+    assert bench._r(0.93817, 3) == 0.938
+    assert bench._r(0.0) == 0.0 and bench._r(None) is None
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    # the CPU oracle arm on the tiny workload: measured per-step time, the same
+    # config object as the GPU arm, the CPU model recorded
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "3",
+                             "--warmup", "1", "--cpu-seconds", "1.5"])
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    from grouped_gemm_plan_b200 import workload as W
+    assert line["impl"] == "reference" and line["steps"] == 3
+    assert line["config"] == bench.workload_config(W.WORKLOADS["tiny"], 1)
+    per_step_s = line["ms_per_step"] / 1e3
+    assert 0.0 < per_step_s < 5.0                      # measured, not extrapolated
+    assert abs(line["tokens_per_step"] / per_step_s - line["value"]) <= 0.05 * line["value"]
+    assert line["ms_per_full_batch_extrapolated"] >= line["ms_per_step"] * 0.99
+    assert line["cpu_baseline"]["cpu_model"] and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

@@ -168,16 +168,34 @@ def test_stage_events(cuda_dev, n_c):
     assert evs[0].elapsed_time(evs[5]) == total
 
 
-def _sample_tokens(ids, n, seed):
-    """First, last and random tokens, plus one token of the heaviest and lightest expert."""
-    M = ids.shape[0]
+def _sample_tokens(ids, perm, offsets, n, seed):
+    """Tokens whose output rows are compared with the oracle at full size.
+
+    Every expert's first and last slot; for the heaviest and the lightest expert
+    the slots on both sides of every 128-row and 256-row m-tile boundary (the
+    single-CTA and the CTA-pair kernels' tiles); the first and last token; then
+    random tokens until there are n (or all M).
+    """
+    M, topk = ids.shape
     rng = np.random.default_rng(seed)
-    counts = np.bincount(ids.reshape(-1))
+    counts = np.diff(offsets)
     picks = {0, M - 1}
+
+    def slot_token(s):
+        picks.add(int(perm[s]) // topk)
+
     nz = np.flatnonzero(counts)
-    for e in (nz[np.argmax(counts[nz])], nz[np.argmin(counts[nz])]):
-        picks.add(int(np.flatnonzero((ids == e).any(1))[0]))
-    picks.update(rng.choice(M, size=min(M, n), replace=False).tolist())
+    for e in nz:
+        slot_token(offsets[e])
+        slot_token(offsets[e + 1] - 1)
+    for e in {int(nz[np.argmax(counts[nz])]), int(nz[np.argmin(counts[nz])])}:
+        for bm in (128, 256):
+            for b in range(bm, int(counts[e]), bm):
+                slot_token(offsets[e] + b - 1)
+                slot_token(offsets[e] + b)
+    rest = np.setdiff1d(np.arange(M), np.fromiter(picks, np.int64))
+    extra = max(0, min(n, M) - len(picks))
+    picks.update(rng.choice(rest, size=min(extra, rest.size), replace=False).tolist())
     return np.array(sorted(picks), np.int64)
 
 
@@ -195,7 +213,8 @@ def test_workload_full_size(cuda_dev, name):
     assert np.array_equal(counts.cpu().numpy(), rc)
     assert np.array_equal(offsets.cpu().numpy(), ro)
     assert np.array_equal(perm.cpu().numpy(), rp)
-    tokens = _sample_tokens(ids, 12, w.seed)
+    tokens = _sample_tokens(ids, rp, ro, 256, w.seed)
+    assert tokens.size >= min(256, w.M)
     W1c, W2c = W1.cpu(), W2.cpu()
     ref_rows = oracle.bruteforce_tokens(x, W1c, W2c, ids, tw, tokens)
     check_close(out.cpu()[torch.from_numpy(tokens)], ref_rows, f"{name} sampled rows")
