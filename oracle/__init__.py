@@ -52,6 +52,7 @@ def configure(lib):
     lib.oracle_bruteforce_tokens.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P]
     lib.oracle_bruteforce_tokens.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_gemm_add.argtypes = [P, P, ctypes.c_double, ctypes.c_double, i64, P]
     lib.oracle_route.argtypes = [P, i64, i32, i32, P, P]
     lib.oracle_route.restype = ctypes.c_int
     lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -193,6 +194,22 @@ def moe_ffn(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
     if st != OK:
         raise OracleError(f"oracle_moe_ffn status {st}")
     return out
+
+
+def gemm_add(acc: np.ndarray, add, alpha: float, beta: float) -> np.ndarray:
+    """alpha * acc + beta * add in fp64 (the Fused GemmAdd epilogue); acc fp64, add bf16."""
+    a = np.ascontiguousarray(acc, dtype=np.float64)
+    b = _u16(add)
+    assert a.shape == b.shape
+    y = np.empty_like(a)
+    _load().oracle_gemm_add(_p(a), _p(b), float(alpha), float(beta), a.size, _p(y))
+    return y
+
+
+def moe_ffn_add(x, W1, W2, ids: np.ndarray, w: np.ndarray, add, alpha: float = 1.0,
+                beta: float = 1.0) -> np.ndarray:
+    """The layer with the GemmAdd epilogue: alpha * layer(x) + beta * add (fp64)."""
+    return gemm_add(moe_ffn(x, W1, W2, ids, w), add, alpha, beta)
 
 
 def route(logits: np.ndarray, topk: int):

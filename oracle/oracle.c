@@ -46,6 +46,9 @@
  *   fp8 GEMM        numpy float64 matmul of the decoded operands
  *   fp8 layer       E=1,topk=1 equals torch's dense chain with the same
  *                   quantisation; within the e4m3 error bound of the exact layer
+ *   gemm add        beta = 0 and alpha = 0 reduce to the layer and to the added
+ *                   tensor exactly; (out - add) of the residual form equals the
+ *                   layer; linear in alpha and beta
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -290,6 +293,21 @@ done:
     free(xp);
     free(yp);
     return st;
+}
+
+/*
+ * Fused GemmAdd epilogue (grouped GEMM article, section "Fused GemmAdd"): the
+ * accumulated result and an added tensor combined before the one output cast,
+ *   y[i] = alpha * acc[i] + beta * add[i]
+ * here applied to the layer output: acc fp64 [n] (e.g. oracle_moe_ffn's out),
+ * add bf16 [n] (e.g. the residual stream x), y fp64 [n].  Nothing is rounded.
+ */
+void oracle_gemm_add(const double *acc, const uint16_t *add, double alpha, double beta, int64_t n,
+                     double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++)
+        y[i] = alpha * acc[i] + beta * bf16_widen(add[i]);
 }
 
 /*

@@ -44,6 +44,10 @@ MUTANTS = {
                           "float sc = amax > 0.0f ? amax / 240.0f : 1.0f;\n        scale[r] = sc;"),
     "fp8_cols_not_transposed": ("qrow[k] = oracle_e4m3_encode((float)bf16_widen(Be[k * N + n]) / sc);",
                                 "qrow[k] = oracle_e4m3_encode((float)bf16_widen(Be[n * K + k]) / sc);"),
+    "gemm_add_alpha_beta_swapped": ("y[i] = alpha * acc[i] + beta * bf16_widen(add[i]);",
+                                    "y[i] = beta * acc[i] + alpha * bf16_widen(add[i]);"),
+    "gemm_add_drops_add": ("y[i] = alpha * acc[i] + beta * bf16_widen(add[i]);",
+                           "y[i] = alpha * acc[i];"),
     "fp8_gemm_drops_b_scale": ("C[s * N + n] = (double)a_scale[s] * (double)b_scale[(int64_t)e * N + n] * acc;",
                                "C[s * N + n] = (double)a_scale[s] * acc;"),
 }
@@ -77,6 +81,8 @@ CHILD = textwrap.dedent("""
         pins.test_layer_matches_torch_per_token_mixture,
         pins.test_route_matches_lexsort_and_softmax,
         pins.test_route_closed_form_and_permutation_equivariance,
+        pins.test_gemm_add_special_cases,
+        pins.test_gemm_add_linear_in_alpha_and_beta,
     ]
     caught = 0
     for c in calls:

@@ -290,3 +290,42 @@ def test_route_closed_form_and_permutation_equivariance():
 def test_route_rejects_topk_above_e():
     with pytest.raises(oracle.OracleError):
         oracle.route(np.zeros((2, 3), np.float32), 4)
+
+
+# ----------------------------------------------------------------------------- GemmAdd
+
+def _gemm_add_case(seed=5):
+    from helpers import layer_case
+    w, x, W1, W2, ids, tw = layer_case(24, 64, 64, 4, 2, "uniform", seed=seed)
+    rng = np.random.default_rng(seed)
+    add = torch.from_numpy(rng.standard_normal((24, 64)).astype(np.float32)).to(torch.bfloat16)
+    return x, W1, W2, ids, tw, add
+
+
+def test_gemm_add_special_cases():
+    """Grouped GEMM article, "Fused GemmAdd": y = alpha * acc + beta * add.  beta = 0
+    is the layer itself, alpha = 0 the added tensor alone (both exact in fp64), and
+    the residual form (alpha = beta = 1) minus the added tensor is the layer."""
+    x, W1, W2, ids, tw, add = _gemm_add_case()
+    layer = oracle.moe_ffn(x, W1, W2, ids, tw)
+    add64 = add.double().numpy()
+    assert np.array_equal(oracle.moe_ffn_add(x, W1, W2, ids, tw, add, 1.0, 0.0), layer)
+    assert np.array_equal(oracle.moe_ffn_add(x, W1, W2, ids, tw, add, 0.0, 1.0), add64)
+    assert np.array_equal(oracle.moe_ffn_add(x, W1, W2, ids, tw, add, 2.0, 0.0), 2.0 * layer)
+    res = oracle.moe_ffn_add(x, W1, W2, ids, tw, add)             # alpha = beta = 1
+    scale = np.abs(layer) + np.abs(add64)
+    assert np.all(np.abs((res - add64) - layer) <= 4 * np.finfo(np.float64).eps * scale)
+    # the residual stream as the added tensor: x + layer(x)
+    resx = oracle.moe_ffn_add(x, W1, W2, ids, tw, x)
+    assert np.all(np.abs(resx - x.double().numpy() - layer) <=
+                  4 * np.finfo(np.float64).eps * (np.abs(layer) + np.abs(x.double().numpy())))
+
+
+def test_gemm_add_linear_in_alpha_and_beta():
+    x, W1, W2, ids, tw, add = _gemm_add_case(seed=6)
+    layer = oracle.moe_ffn(x, W1, W2, ids, tw)
+    add64 = add.double().numpy()
+    for alpha, beta in [(0.5, -2.0), (-1.0, 0.25), (3.0, 3.0)]:
+        y = oracle.moe_ffn_add(x, W1, W2, ids, tw, add, alpha, beta)
+        ref = alpha * layer + beta * add64          # numpy on the two pinned parts
+        assert np.allclose(y, ref, rtol=1e-14, atol=1e-14)
