@@ -30,7 +30,8 @@ OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FF
 
 # Every symbol include/moe.h declares.
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_plan", "moe_dispatch",
-           "moe_grouped_gemm", "moe_combine", "moe_ffn_fused", "moe_ffn_fused_noalloc",
+           "moe_grouped_gemm", "moe_combine", "moe_combine_add", "moe_ffn_fused",
+           "moe_ffn_fused_add", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
            "moe_set_stage_events", "moe_quantize_weights_e4m3", "moe_quantize_rows_e4m3",
            "moe_grouped_gemm_e4m3", "moe_ffn_fused_fp8", "moe_last_error"]
@@ -76,6 +77,12 @@ def load(path: str | None = None):
     lib.moe_combine.restype = st
     lib.moe_ffn_fused.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]
     lib.moe_ffn_fused.restype = st
+    f32 = ctypes.c_float
+    lib.moe_combine_add.argtypes = [P, i32, P, P, P, f32, f32, i64, i64, i32, P, P, sz, P]
+    lib.moe_combine_add.restype = st
+    lib.moe_ffn_fused_add.argtypes = [P, P, P, P, P, P, f32, f32, i64, i64, i64, i32, i32, P, P,
+                                      P, P, P, sz, P]
+    lib.moe_ffn_fused_add.restype = st
     lib.moe_ffn_fused_noalloc.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P, P]
     lib.moe_ffn_fused_noalloc.restype = st
     lib.moe_get_device_status.argtypes = [P, P]
@@ -184,6 +191,28 @@ def moe_ffn_fused(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, ws, n
     _check(load().moe_ffn_fused(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w), M, H,
                                 F2 // 2, E, topk, n_c, _ptr(out), _ptr(counts), _ptr(offsets),
                                 _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_combine_add(y, inv_perm, topk_w, add, alpha, beta, M, topk, out, ws, stream=None):
+    """moe_combine with the GemmAdd epilogue: out = bf16(alpha * sum + beta * add)."""
+    H = y.shape[1]
+    if y.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("moe_combine_add takes bf16 or fp32 rows")
+    _check(load().moe_combine_add(_ptr(y), 1 if y.dtype == torch.float32 else 0, _ptr(inv_perm),
+                                  _ptr(topk_w), _ptr(add), float(alpha), float(beta), M, H, topk,
+                                  _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_ffn_fused_add(x, W1, W2, topk_ids, topk_w, add, alpha, beta, out, counts, offsets, perm,
+                      ws, stream=None):
+    """The layer with the GemmAdd epilogue: out = bf16(alpha * layer(x) + beta * add)."""
+    M, H = x.shape
+    E, _, F2 = W1.shape
+    topk = topk_ids.shape[1]
+    _check(load().moe_ffn_fused_add(_ptr(x), _ptr(W1), _ptr(W2), _ptr(topk_ids), _ptr(topk_w),
+                                    _ptr(add), float(alpha), float(beta), M, H, F2 // 2, E, topk,
+                                    _ptr(out), _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(ws),
+                                    ws.numel(), _stream(stream)))
 
 
 def moe_ffn_fused_noalloc(x, W1, W2, topk_ids, topk_w, out, counts, offsets, perm, status=None,

@@ -28,6 +28,10 @@ int launch_grouped_gemm(const void* A, const void* B, const int32_t* offsets, in
                         int64_t R, int64_t K, int64_t N, int epi, const float* w_sorted,
                         const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                         int num_sms, cudaStream_t stream);
+cudaError_t launch_combine_add(const void* y, bool y_f32, const int32_t* inv, const float* w,
+                               const void* add, float alpha, float beta, int64_t M, int64_t H,
+                               int32_t topk, void* out, int32_t* status, int num_sms,
+                               cudaStream_t stream);
 size_t layer_sync_bytes(int64_t M, int64_t R, int32_t E);
 cudaError_t launch_quantize_rows(const void* A, int64_t R, int64_t K, void* q, float* scale,
                                  int num_sms, cudaStream_t stream);
@@ -326,6 +330,29 @@ moe_status moe_combine(const void* y, int32_t y_fp32, const int32_t* inv_perm,
   return MOE_OK;
 }
 
+moe_status moe_combine_add(const void* y, int32_t y_fp32, const int32_t* inv_perm,
+                           const float* topk_w, const void* add, float alpha, float beta,
+                           int64_t M, int64_t H, int32_t topk, void* out, void* ws,
+                           size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (M < 0 || topk < 1 || topk > 32 || M > kMaxRows / topk)
+    return fail(MOE_ERR_INVALID_ARG, "bad M=%lld or topk=%d", (long long)M, topk);
+  if (H <= 0 || H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H = %lld must be a positive multiple of 8", (long long)H);
+  moe_status st = check_ws(MOE_OP_COMBINE, ws, ws_bytes, M, H, 0, 1, topk);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  if (y == nullptr || out == nullptr) return fail(MOE_ERR_INVALID_ARG, "y and out must not be NULL");
+  if (add == nullptr && beta != 0.0f) return fail(MOE_ERR_INVALID_ARG, "add is NULL but beta != 0");
+  if (!aligned16(y) || !aligned16(out) || !aligned16(add))
+    return fail(MOE_ERR_MISALIGNED, "y, out and add must be 16-byte aligned");
+  if (y_fp32 != 0 && y_fp32 != 1) return fail(MOE_ERR_INVALID_ARG, "y_fp32 must be 0 or 1");
+  cudaError_t err = moe::launch_combine_add(y, y_fp32 != 0, inv_perm, topk_w, add, alpha, beta,
+                                            M, H, topk, out, status_word(ws), num_sms_current(),
+                                            reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_combine_add launch");
+  return MOE_OK;
+}
+
 moe_status moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets, int32_t E,
                             int64_t R, int64_t K, int64_t N, moe_epilogue epi,
                             const float* w_sorted, const int32_t* perm, void* C, void* ws,
@@ -357,11 +384,18 @@ moe_status moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets
   return MOE_OK;
 }
 
-moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
-                         const float* topk_w, int64_t M, int64_t H, int64_t F, int32_t E,
-                         int32_t topk, int32_t n_c, void* out, int32_t* counts,
-                         int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
-                         void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer (moe_ffn_fused and moe_ffn_fused_add).  n_c as moe_ffn_fused; the
+// combine applies out = bf16(alpha * sum + beta * add) (alpha = 1, beta = 0: the
+// plain layer, add unused).
+moe_status ffn_fused_impl(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
+                          const float* topk_w, const void* add, float alpha, float beta,
+                          int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk, int32_t n_c,
+                          void* out, int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
+                          size_t ws_bytes, void* stream) {
   g_last_error.clear();
   moe_status st = moe::check_layer_shape(M, H, F, E, topk);
   if (st != MOE_OK) return st;
@@ -382,6 +416,10 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
     return fail(MOE_ERR_INVALID_ARG, "x, W1, W2, topk_ids, topk_w, out and perm must not be NULL");
   if (!aligned16(x) || !aligned16(W1) || !aligned16(W2) || !aligned16(out))
     return fail(MOE_ERR_MISALIGNED, "x, W1, W2 and out must be 16-byte aligned");
+  const bool gemm_add = alpha != 1.0f || beta != 0.0f;
+  if (gemm_add && beta != 0.0f && add == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "add is NULL but beta != 0");
+  if (gemm_add && !aligned16(add)) return fail(MOE_ERR_MISALIGNED, "add must be 16-byte aligned");
 
   const int64_t R = M * topk;
   // Overlapping kernel boundaries pays off on small layers only (measured).
@@ -403,7 +441,7 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
                                      perm, inv, w_sorted, status, plan_scratch(ws), sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused plan");
   stage_mark(1, s);
-  const int32_t nc = n_c < 0 ? moe::profiled_n_c(M, H, F, E, topk) : n_c;
+  const int32_t nc = gemm_add ? 0 : (n_c < 0 ? moe::profiled_n_c(M, H, F, E, topk) : n_c);
   if (nc > 0) {
     // One persistent kernel: nc memory CTAs (dispatch, combine) beside the GEMM CTAs.
     if (nc > 64 || nc >= sms) return fail(MOE_ERR_INVALID_ARG, "n_c = %d must be < min(65, #SMs = %d)", nc, sms);
@@ -429,10 +467,33 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
   if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM2)")
                               : cuda_fail(cudaGetLastError(), "moe_ffn_fused GEMM2");
   stage_mark(4, s);
-  err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
+  err = moe::launch_combine_add(yk, true, nullptr, nullptr, add, alpha, beta, M, H, topk, out,
+                                status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused combine");
   stage_mark(5, s);
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const int32_t* topk_ids,
+                         const float* topk_w, int64_t M, int64_t H, int64_t F, int32_t E,
+                         int32_t topk, int32_t n_c, void* out, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                         void* stream) {
+  return ffn_fused_impl(x, W1, W2, topk_ids, topk_w, nullptr, 1.0f, 0.0f, M, H, F, E, topk, n_c,
+                        out, counts, offsets, perm, ws, ws_bytes, stream);
+}
+
+moe_status moe_ffn_fused_add(const void* x, const void* W1, const void* W2,
+                             const int32_t* topk_ids, const float* topk_w, const void* add,
+                             float alpha, float beta, int64_t M, int64_t H, int64_t F, int32_t E,
+                             int32_t topk, void* out, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  return ffn_fused_impl(x, W1, W2, topk_ids, topk_w, add, alpha, beta, M, H, F, E, topk, 0, out,
+                        counts, offsets, perm, ws, ws_bytes, stream);
 }
 
 moe_status moe_quantize_weights_e4m3(const void* W, int32_t E, int64_t K, int64_t N, void* Wq,

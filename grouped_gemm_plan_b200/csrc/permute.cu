@@ -144,13 +144,24 @@ struct Vec8<true> {
   }
 };
 
-// out[t] = bf16(sum_k w[t,k] * y[row(t,k)]), row(t,k) = inv ? inv[t*topk+k] : t*topk+k.
-// y is bf16 or fp32 [R, H]; vpr = H / 8 groups of eight elements per row.
-template <int KMAX, bool F32>
+// Optional epilogue of the combine (the grouped GEMM article's "Fused GemmAdd":
+// the accumulated fp32 result and an fp32 add are combined before the one cast):
+// out[t] = bf16(alpha * acc + beta * add[t]); add is read only when beta != 0.
+struct CombineAdd {
+  const uint4* add;  // bf16 [M, H] (may be the layer's x, or out itself)
+  float alpha, beta;
+};
+
+// out[t] = bf16(sum_k w[t,k] * y[row(t,k)]), row(t,k) = inv ? inv[t*topk+k] : t*topk+k,
+// or with an added tensor bf16(alpha * sum + beta * add[t]).
+// y is bf16 or fp32 [R, H]; vpr = H / 8 groups of eight elements per row.  Each
+// output vector is written by the lane that read its add vector, so add may
+// alias out.
+template <int KMAX, bool F32, bool ADD>
 __global__ void __launch_bounds__(PM_THREADS)
     combine_kernel(const uint8_t* __restrict__ y, const int32_t* __restrict__ inv,
                    const float* __restrict__ w, int32_t M, int32_t R, int32_t topk,
-                   int32_t vpr, uint4* __restrict__ out, int32_t* status) {
+                   int32_t vpr, uint4* out, int32_t* status, CombineAdd ga) {
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
@@ -214,6 +225,19 @@ __global__ void __launch_bounds__(PM_THREADS)
     for (int u = 0; u < CU; ++u) {
       const int32_t c = cbase + 32 * u;
       if (c >= vpr) continue;
+      if (ADD) {
+        if (ga.beta != 0.0f) {
+          const uint4 a = ga.add[static_cast<int64_t>(t) * vpr + c];
+          const float2 a0 = unpack_bf16x2(a.x), a1 = unpack_bf16x2(a.y), a2 = unpack_bf16x2(a.z),
+                       a3 = unpack_bf16x2(a.w);
+          const float av[8] = {a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[u][e] = fmaf(ga.beta, av[e], ga.alpha * acc[u][e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[u][e] *= ga.alpha;
+        }
+      }
       uint4 o;
       o.x = pack_bf16x2(acc[u][0], acc[u][1]);
       o.y = pack_bf16x2(acc[u][2], acc[u][3]);
@@ -253,27 +277,27 @@ cudaError_t launch_dispatch_tokens(const void* x, const int32_t* inv, int64_t M,
                     reinterpret_cast<uint4*>(xp), status);
 }
 
-template <bool F32>
+template <bool F32, bool ADD>
 static cudaError_t launch_combine_t(int grid, cudaStream_t stream, const uint8_t* y, const int32_t* inv,
-                             const float* w, int32_t m, int32_t R, int32_t topk, int32_t vpr,
-                             uint4* ov, int32_t* status) {
-  cudaError_t err;
+                                    const float* w, int32_t m, int32_t R, int32_t topk, int32_t vpr,
+                                    uint4* ov, int32_t* status, CombineAdd ga) {
+  const dim3 g(grid), b(PM_THREADS);
   if (topk <= 2)
-    err = launch_pdl(combine_kernel<2, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 4)
-    err = launch_pdl(combine_kernel<4, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 8)
-    err = launch_pdl(combine_kernel<8, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
-  else if (topk <= 16)
-    err = launch_pdl(combine_kernel<16, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
-  else
-    err = launch_pdl(combine_kernel<32, F32>, dim3(grid), dim3(PM_THREADS), 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status);
-  return err;
+    return launch_pdl(combine_kernel<2, F32, ADD>, g, b, 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status, ga);
+  if (topk <= 4)
+    return launch_pdl(combine_kernel<4, F32, ADD>, g, b, 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status, ga);
+  if (topk <= 8)
+    return launch_pdl(combine_kernel<8, F32, ADD>, g, b, 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status, ga);
+  if (topk <= 16)
+    return launch_pdl(combine_kernel<16, F32, ADD>, g, b, 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status, ga);
+  return launch_pdl(combine_kernel<32, F32, ADD>, g, b, 0, stream, 1, y, inv, w, m, R, topk, vpr, ov, status, ga);
 }
 
-cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
-                           int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
-                           int num_sms, cudaStream_t stream) {
+// alpha == 1 and beta == 0: the plain combine (add unused, may be nullptr).
+cudaError_t launch_combine_add(const void* y, bool y_f32, const int32_t* inv, const float* w,
+                               const void* add, float alpha, float beta, int64_t M, int64_t H,
+                               int32_t topk, void* out, int32_t* status, int num_sms,
+                               cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   const int grid = grid_for_items(M * ((H / 8 + 31) / 32), num_sms);
   const int32_t R = static_cast<int32_t>(M * topk);
@@ -281,8 +305,19 @@ cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const 
   const uint8_t* yb = reinterpret_cast<const uint8_t*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out);
   const int32_t m = static_cast<int32_t>(M);
-  return y_f32 ? launch_combine_t<true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status)
-               : launch_combine_t<false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status);
+  const CombineAdd ga{reinterpret_cast<const uint4*>(add), alpha, beta};
+  if (alpha != 1.0f || beta != 0.0f)
+    return y_f32 ? launch_combine_t<true, true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status, ga)
+                 : launch_combine_t<false, true>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status, ga);
+  return y_f32 ? launch_combine_t<true, false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status, ga)
+               : launch_combine_t<false, false>(grid, stream, yb, inv, w, m, R, topk, vpr, ov, status, ga);
+}
+
+cudaError_t launch_combine(const void* y, bool y_f32, const int32_t* inv, const float* w,
+                           int64_t M, int64_t H, int32_t topk, void* out, int32_t* status,
+                           int num_sms, cudaStream_t stream) {
+  return launch_combine_add(y, y_f32, inv, w, nullptr, 1.0f, 0.0f, M, H, topk, out, status, num_sms,
+                            stream);
 }
 
 }  // namespace moe

@@ -77,6 +77,12 @@ WORKLOADS: dict[str, Workload] = {
     # profiling size: the Mixtral expert shape with two experts (0.7 GB of weights,
     # still far above L2), used for single-kernel hardware-counter captures
     "mixtral_prof": Workload("mixtral_prof", 2048, 4096, 14336, 2, 2, "balanced", 0.0, 101),
+    # the Qwen2-MoE expert shape and load with 16 of its 64 experts (and a quarter of
+    # its tokens, so experts keep their rows): 0.28 GB of weights, above L2
+    "qwen2_prof": Workload("qwen2_prof", 2048, 2048, 1408, 16, 4, "skewed", 0.032, 202),
+    # the Phi-3.5-MoE expert shape with 4 of its 16 experts, 4096 rows each
+    # (balanced): 0.63 GB of weights; x and the dispatched rows (0.2 GB) above L2
+    "phi35_prof": Workload("phi35_prof", 8192, 4096, 6400, 4, 2, "balanced", 0.0, 303),
 }
 
 

@@ -205,6 +205,40 @@ moe_status moe_ffn_fused(const void* x, const void* W1, const void* W2, const in
                          int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
                          void* stream);
 
+/*
+ * moe_combine_add -- moe_combine with the Fused GemmAdd epilogue ([GG] "Fused
+ * GemmAdd": Y = cast(alpha * Acc_fp32 + beta * Add_fp32), the addition done in
+ * fp32 before the one cast):
+ *   out[t, :] = bf16( alpha * sum_k wk * fp32(y[row(t, k), :]) + beta * fp32(add[t, :]) )
+ * with row(t, k), wk, y and y_fp32 as in moe_combine; add bf16 [M, H] (e.g. the
+ * residual stream), 16-byte aligned.  add is read only when beta != 0 (it may
+ * then be NULL); add may be the same buffer as out.  alpha = 1 and beta = 0
+ * give exactly moe_combine's result.
+ */
+moe_status moe_combine_add(const void* y, int32_t y_fp32, const int32_t* inv_perm,
+                           const float* topk_w, const void* add, float alpha, float beta,
+                           int64_t M, int64_t H, int32_t topk, void* out, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * moe_ffn_fused_add -- the layer with the Fused GemmAdd epilogue ([GG] "Fused
+ * GemmAdd"), e.g. the residual connection around the MoE layer:
+ *   out[t, :] = bf16( alpha * sum_k topk_w[t, k] * FFN_{topk_ids[t, k]}(x[t, :])
+ *                     + beta * add[t, :] )
+ * The addition happens in fp32 inside the combine, before the single bf16 cast
+ * (no extra pass over out).  add bf16 [M, H], read only when beta != 0; it may be
+ * x itself (out = x + layer(x) with alpha = beta = 1) or the same buffer as out.
+ * Other arguments, the workspace (moe_workspace_size(MOE_OP_FFN_FUSED, ...)) and
+ * the errors are those of moe_ffn_fused; the stages run as consecutive kernels
+ * (as moe_ffn_fused with n_c = 0).  alpha = 1 and beta = 0 give exactly
+ * moe_ffn_fused's result.
+ */
+moe_status moe_ffn_fused_add(const void* x, const void* W1, const void* W2,
+                             const int32_t* topk_ids, const float* topk_w, const void* add,
+                             float alpha, float beta, int64_t M, int64_t H, int64_t F, int32_t E,
+                             int32_t topk, void* out, int32_t* counts, int32_t* offsets,
+                             int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
 /* Size of the library's own device scratch used by moe_ffn_fused_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 

@@ -135,6 +135,27 @@ def test_fused_validation(lib):
     assert f(*args(ws=need - 1)) == 4
 
 
+def test_gemm_add_validation(lib):
+    # moe_combine_add: beta != 0 needs the added tensor; it must be 16-byte aligned
+    ca = lib.moe_combine_add
+    assert ca(FAKE, 0, FAKE, FAKE, None, 1.0, 1.0, 4, 64, 2, FAKE, FAKE_WS, 256, None) == 1
+    assert ca(FAKE, 0, FAKE, FAKE, ctypes.c_void_p(0x10004), 1.0, 1.0, 4, 64, 2, FAKE, FAKE_WS,
+              256, None) == 7
+    assert ca(FAKE, 0, FAKE, FAKE, FAKE, 1.0, 1.0, 4, 100, 2, FAKE, FAKE_WS, 256, None) == 2
+    assert ca(None, 0, None, None, None, 1.0, 1.0, 0, 64, 2, None, FAKE_WS, 256, None) == 0
+    # moe_ffn_fused_add: the layer's checks, then the added tensor's
+    fa = lib.moe_ffn_fused_add
+    need = B.moe_workspace_size(B.OP_FFN_FUSED, 16, 128, 128, 4, 2)
+    args = lambda **kw: [FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("add", FAKE), kw.get("alpha", 1.0),
+                         kw.get("beta", 1.0), 16, kw.get("H", 128), 128, 4, 2, FAKE, FAKE, FAKE,
+                         FAKE, FAKE_WS, kw.get("ws", need), None]
+    assert fa(*args(H=100)) == 2
+    assert fa(*args(add=None)) == 1
+    assert "add is NULL" in B.moe_last_error()
+    assert fa(*args(add=ctypes.c_void_p(0x10004))) == 7
+    assert fa(*args(ws=need - 1)) == 4
+
+
 def test_fp8_validation(lib):
     qw = lib.moe_quantize_weights_e4m3
     assert qw(FAKE, 0, 64, 64, FAKE, FAKE, None) == 2               # E

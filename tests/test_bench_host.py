@@ -62,7 +62,7 @@ def test_default_arguments():
     assert (a.gpus, a.steps, a.warmup, a.impl, a.workload) == (1, 20, 5, "ours", "phi35")
     assert a.warmup >= 3 and a.side_warmup >= 3
     from grouped_gemm_plan_b200 import workload as W
-    flops = {n: W.WORKLOADS[n].flops() for n in W.WORKLOADS if n != "mixtral_prof"}
+    flops = {n: W.WORKLOADS[n].flops() for n in W.WORKLOADS if not n.endswith("_prof")}
     assert max(flops, key=flops.get) == a.workload
     assert set(a.side.split(",")) | {a.workload} == set(flops)
 
