@@ -216,42 +216,54 @@ __global__ void __launch_bounds__(PLAN_THREADS)
   }
 }
 
-// Host launcher (no validation here; the C ABI layer validates).  `scratch`
-// holds plan_hist_rows(E) ints (the per-chunk histograms).
-cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
-                        int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
-                        int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream) {
-  const size_t smem = sizeof(int32_t) * (size_t)(2 + PLAN_WARPS) * (size_t)E;
+// Rows each warp of the plan kernel owns for R routed rows (a multiple of 32):
+// the rows are cut into at most min(#SMs, 256) chunks of 16 warps.
+int32_t plan_warp_rows(int32_t R, int num_sms) {
+  const int max_chunks = num_sms < PLAN_MAX_CHUNKS ? num_sms : PLAN_MAX_CHUNKS;
+  const int32_t per_cta = (R + max_chunks - 1) / max_chunks;
+  int32_t seg = (per_cta + PLAN_WARPS - 1) / PLAN_WARPS;
+  seg = ((seg + 31) / 32) * 32;
+  return seg < 32 ? 32 : seg;
+}
+
+// The scan-and-scatter kernel over `nchunks` chunks of 16 * seg rows, from the
+// per-chunk histograms `hist` (nullptr: one chunk that counts its own rows).
+cudaError_t launch_plan_chunks(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t seg,
+                               const int32_t* hist, int32_t nchunks, int32_t* counts,
+                               int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
+                               int32_t* status, cudaStream_t stream) {
   static PerDeviceOnce once;
   const cudaError_t aerr = once.run([] {
     return cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(sizeof(int32_t) * (2 + PLAN_WARPS) * MOE_MAX_EXPERTS));
   });
   if (aerr != cudaSuccess) return aerr;
-  if (R == 0) {
-    // Only counts/offsets to write: one CTA with no rows.
-    return launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), smem, stream, 1, ids, w, 0, E, 32,
-                      static_cast<const int32_t*>(nullptr), 0, counts, offsets, perm, inv, w_sorted,
-                      status);
-  }
-  const int max_chunks = num_sms < PLAN_MAX_CHUNKS ? num_sms : PLAN_MAX_CHUNKS;
-  int32_t per_cta = (R + max_chunks - 1) / max_chunks;
-  int32_t seg = (per_cta + PLAN_WARPS - 1) / PLAN_WARPS;
-  seg = ((seg + 31) / 32) * 32;
-  if (seg < 32) seg = 32;
+  const size_t smem = sizeof(int32_t) * (size_t)(2 + PLAN_WARPS) * (size_t)E;
+  const int32_t grid = hist == nullptr ? 1 : nchunks;
+  return launch_pdl(plan_kernel, dim3(grid), dim3(PLAN_THREADS), smem, stream, 1, ids, w, R, E, seg,
+                    hist, hist == nullptr ? 1 : nchunks, counts, offsets, perm, inv, w_sorted,
+                    status);
+}
+
+// Host launcher (no validation here; the C ABI layer validates).  `scratch`
+// holds the per-chunk histograms (256 x (E + 1) ints).
+cudaError_t launch_plan(const int32_t* ids, const float* w, int32_t R, int32_t E, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, float* w_sorted,
+                        int32_t* status, int32_t* scratch, int num_sms, cudaStream_t stream) {
+  if (R == 0)  // only counts/offsets to write: one CTA with no rows
+    return launch_plan_chunks(ids, w, 0, E, 32, nullptr, 0, counts, offsets, perm, inv, w_sorted,
+                              status, stream);
+  const int32_t seg = plan_warp_rows(R, num_sms);
   const int32_t chunk = seg * PLAN_WARPS;
   const int32_t grid = (R + chunk - 1) / chunk;
-  if (grid == 1) {
-    return launch_pdl(plan_kernel, dim3(1), dim3(PLAN_THREADS), smem, stream, 1, ids, w, R, E, seg,
-                      static_cast<const int32_t*>(nullptr), 1, counts, offsets, perm, inv, w_sorted,
-                      status);
-  }
+  if (grid == 1)
+    return launch_plan_chunks(ids, w, R, E, seg, nullptr, 1, counts, offsets, perm, inv, w_sorted,
+                              status, stream);
   cudaError_t err = launch_pdl(plan_hist_kernel, dim3(grid), dim3(PLAN_THREADS), sizeof(int32_t) * E,
                                stream, 1, ids, R, E, seg, scratch);
   if (err != cudaSuccess) return err;
-  return launch_pdl(plan_kernel, dim3(grid), dim3(PLAN_THREADS), smem, stream, 1, ids, w, R, E, seg,
-                    static_cast<const int32_t*>(scratch), grid, counts, offsets, perm, inv, w_sorted,
-                    status);
+  return launch_plan_chunks(ids, w, R, E, seg, scratch, grid, counts, offsets, perm, inv, w_sorted,
+                            status, stream);
 }
 
 }  // namespace moe
