@@ -325,10 +325,9 @@ def plan_launches(R: int, num_sms: int) -> int:
 
 
 def gemm_uses_pair(R: int, E: int) -> bool:
-    """Which GEMM kernel the library runs for this shape (its rule: CTA pairs once
-    experts average 1024 rows or more, unless MOE_GEMM_PAIR forces one)."""
-    forced = os.environ.get("MOE_GEMM_PAIR", "")
-    return forced == "1" or (forced != "0" and R >= 1024 * E)
+    """Which bf16 GEMM kernel the library runs (its rule: CTA pairs unless
+    MOE_GEMM_PAIR=0 forces the single-CTA kernel)."""
+    return os.environ.get("MOE_GEMM_PAIR", "") != "0" and R > 0 and E > 0
 
 
 def stage_timing_in_step(wl) -> bool:
@@ -474,21 +473,50 @@ class LayerRun:
                 for j, n in enumerate(self.STAGES)}
 
     def router_us(self):
+        """Device time of the router in front of the layer and of the plan, from CUDA
+        graphs of 20 calls each (no host launch overhead in the figure): moe_route
+        then moe_plan as two calls, and moe_route_plan (the router fused with the
+        plan's histogram pass).  Returns microseconds per call pair / fused call."""
         torch, B, wl, dev = self.torch, self.B, self.wl, self.dev
+        M, E, topk, R = wl.M, wl.E, wl.topk, wl.R
         g = torch.Generator(device=dev).manual_seed(wl.seed)
-        logits = torch.randn((wl.M, wl.E), generator=g, device=dev, dtype=torch.float32)
-        r_ids = torch.empty((wl.M, wl.topk), dtype=torch.int32, device=dev)
-        r_w = torch.empty((wl.M, wl.topk), dtype=torch.float32, device=dev)
-        r_ws = B.alloc_workspace(B.OP_ROUTE, wl.M, 0, 0, wl.E, wl.topk, dev)
-        rev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        B.moe_route(logits, wl.topk, r_ids, r_w, r_ws)
-        rev[0].record(self.stream)
-        for _ in range(10):
-            B.moe_route(logits, wl.topk, r_ids, r_w, r_ws)
-        rev[1].record(self.stream)
-        torch.cuda.synchronize()
-        self.check_status(r_ws, "after the router")
-        return rev[0].elapsed_time(rev[1]) * 100.0
+        logits = torch.randn((M, E), generator=g, device=dev, dtype=torch.float32)
+        r_ids = torch.empty((M, topk), dtype=torch.int32, device=dev)
+        r_w = torch.empty((M, topk), dtype=torch.float32, device=dev)
+        cnt = torch.empty(E, dtype=torch.int32, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(R, dtype=torch.int32, device=dev)
+        inv = torch.empty(R, dtype=torch.int32, device=dev)
+        wsrt = torch.empty(R, dtype=torch.float32, device=dev)
+        ws = B.alloc_workspace(B.OP_PLAN, M, 0, 0, E, topk, dev)
+
+        def separate():
+            B.moe_route(logits, topk, r_ids, r_w, ws)
+            B.moe_plan(r_ids, r_w, E, cnt, off, perm, inv, wsrt, ws)
+
+        def fused():
+            B.moe_route_plan(logits, topk, r_ids, r_w, cnt, off, perm, inv, wsrt, ws)
+
+        out = {}
+        for name, fn in (("route_then_plan_us", separate), ("route_plan_fused_us", fused)):
+            fn()
+            torch.cuda.synchronize()
+            self.check_status(ws, "after the router")
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(20):
+                    fn()
+            graph.replay()
+            ev = self.events(3)
+            for a, b in ev:
+                a.record(self.stream)
+                graph.replay()
+                b.record(self.stream)
+            torch.cuda.synchronize()
+            self.check_status(ws, "after the router graph")
+            out[name] = min(a.elapsed_time(b) for a, b in ev) * 1e3 / 20
+            del graph
+        return out
 
     def fp8_leg(self, steps, warmup):
         """The layer with the FP8 (E4M3) down projection: W2 quantised once
@@ -741,8 +769,9 @@ def run_ours(args):
     achieved = rates["gemm1_tflops"]
     pair = gemm_uses_pair(R, E)
     roofline = {"kernel": "grouped GEMM1 + SwiGLU epilogue",
-                "kernel_variant": ("grouped_gemm_2sm_kernel (CTA pair, 256x256 tiles)" if pair
-                                   else "grouped_gemm_kernel (single CTA, 128x256 tiles)"),
+                "kernel_variant": ("grouped_gemm_2sm_kernel (CTA pairs, device tile queue, "
+                                   "256x256 tiles, 128-row expert tails, N-halves at the end)"
+                                   if pair else "grouped_gemm_kernel (single CTA, 128x256 tiles)"),
                 "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{pk_kind} " + ("bf16_tflops_sustained (SM clock dropped under the "
@@ -803,7 +832,7 @@ def run_ours(args):
             "combine_frac_of_hbm": rates["combine_frac_of_hbm"],
             "hbm_peak_gbs": pk["hbm_gbs"],
             "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
-            "router_us": router_us,
+            "router_plan_us": router_us,
             "fp8_layer": fp8_info,
             # last, so that they stay in view at the end of the line: one record per
             # other workload, columns as named (fractions of the measured burst

@@ -29,7 +29,8 @@ OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FF
     0, 1, 2, 3, 4, 5, 6
 
 # Every symbol include/moe.h declares.
-EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_plan", "moe_dispatch",
+EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_route_plan", "moe_plan",
+           "moe_dispatch",
            "moe_grouped_gemm", "moe_combine", "moe_combine_add", "moe_ffn_fused",
            "moe_ffn_fused_add", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
@@ -67,6 +68,8 @@ def load(path: str | None = None):
     lib.moe_workspace_size.restype = sz
     lib.moe_route.argtypes = [P, i64, i32, i32, P, P, P, sz, P]
     lib.moe_route.restype = st
+    lib.moe_route_plan.argtypes = [P, i64, i32, i32, P, P, P, P, P, P, P, P, sz, P]
+    lib.moe_route_plan.restype = st
     lib.moe_plan.argtypes = [P, P, i64, i32, i32, P, P, P, P, P, P, sz, P]
     lib.moe_plan.restype = st
     lib.moe_dispatch.argtypes = [P, P, i64, i64, i32, P, P, sz, P]
@@ -148,6 +151,16 @@ def moe_route(logits, topk, topk_ids, topk_w, ws, stream=None):
         raise ValueError("moe_route takes fp32 logits")
     _check(load().moe_route(_ptr(logits), M, E, topk, _ptr(topk_ids), _ptr(topk_w), _ptr(ws),
                             ws.numel(), _stream(stream)))
+
+
+def moe_route_plan(logits, topk, topk_ids, topk_w, counts, offsets, perm, inv_perm, w_sorted, ws,
+                   stream=None):
+    M, E = logits.shape
+    if logits.dtype != torch.float32:
+        raise ValueError("moe_route_plan takes fp32 logits")
+    _check(load().moe_route_plan(_ptr(logits), M, E, topk, _ptr(topk_ids), _ptr(topk_w),
+                                 _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+                                 _ptr(w_sorted), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def moe_plan(topk_ids, topk_w, E, counts, offsets, perm, inv_perm, w_sorted, ws, stream=None):

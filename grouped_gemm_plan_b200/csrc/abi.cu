@@ -50,6 +50,10 @@ int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_
 int32_t profiled_n_c(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
 cudaError_t launch_route(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* ids,
                          float* w, int num_sms, cudaStream_t stream);
+cudaError_t launch_route_plan(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* ids,
+                              float* w, int32_t* counts, int32_t* offsets, int32_t* perm,
+                              int32_t* inv, float* w_sorted, int32_t* status, int32_t* scratch,
+                              int num_sms, cudaStream_t stream);
 }  // namespace moe
 
 namespace {
@@ -248,7 +252,8 @@ moe_status moe_get_device_status(void* ws, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int32_t v = 0;
   cudaError_t err = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
-  if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, sizeof v, s);
+  // the whole control block: status word and the GEMM tile queue
+  if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, kCtrlBytes, s);
   if (err == cudaSuccess) err = cudaStreamSynchronize(s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_get_device_status");
   return static_cast<moe_status>(v);
@@ -289,6 +294,27 @@ moe_status moe_route(const float* logits, int64_t M, int32_t E, int32_t topk, in
   cudaError_t err = moe::launch_route(logits, M, E, topk, topk_ids, topk_w, num_sms_current(),
                                       reinterpret_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "moe_route launch");
+  return MOE_OK;
+}
+
+moe_status moe_route_plan(const float* logits, int64_t M, int32_t E, int32_t topk,
+                          int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv_perm, float* w_sorted, void* ws,
+                          size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  moe_status st = check_route(M, E, topk);
+  if (st != MOE_OK) return st;
+  st = check_ws(MOE_OP_PLAN, ws, ws_bytes, M, 0, 0, E, topk);
+  if (st != MOE_OK) return st;
+  if (counts == nullptr || offsets == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  if (M > 0 && (logits == nullptr || topk_ids == nullptr || topk_w == nullptr || perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "logits, topk_ids, topk_w and perm must not be NULL");
+  cudaError_t err = moe::launch_route_plan(logits, M, E, topk, topk_ids, topk_w, counts, offsets,
+                                           perm, inv_perm, w_sorted, status_word(ws),
+                                           plan_scratch(ws), num_sms_current(),
+                                           reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_route_plan launch");
   return MOE_OK;
 }
 

@@ -56,6 +56,60 @@ __device__ __forceinline__ void pack8_swiglu(const float* g, const float* u, uin
   out.w = pack_bf16x2(silu_fast(g[6]) * u[6], silu_fast(g[7]) * u[7]);
 }
 
+// The epilogue of `nseg` 128-byte output segments of this warp's 32 rows:
+//   EPI = MOE_EPI_STORE           segment c: bf16 of accumulator cols [64c, 64c + 64)
+//         MOE_EPI_SWIGLU          segment c: bf16 silu(gate) * up of gate cols
+//                                 [64c, 64c + 64) and up cols up_off + [64c, 64c + 64)
+//         MOE_EPI_WEIGHT_SCATTER  segment c: fp32 of accumulator cols [32c, 32c + 32) * scale
+// t_row: TMEM address of this warp's lanes, first accumulator column; row_dst: byte
+// address of this thread's output row at the warp's first output column (nullptr:
+// the row is not written); n_left: output columns from there to the end of the
+// row (segments past it are skipped).  Warp-collective.
+template <int EPI>
+__device__ __forceinline__ void epilogue_segments(uint32_t t_row, uint8_t* row_dst, int32_t n_left,
+                                                  int nseg, uint32_t up_off, float scale,
+                                                  uint4* buf, int lane) {
+#pragma unroll 1
+  for (int c = 0; c < nseg; ++c) {
+    uint4 seg[8];
+    if (EPI == MOE_EPI_SWIGLU) {
+      float g[32], u[32];
+      tmem_ld32(t_row + c * 64, g);
+      tmem_ld32(t_row + up_off + c * 64, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_swiglu(g + 8 * q, u + 8 * q, seg[q]);
+      tmem_ld32(t_row + c * 64 + 32, g);
+      tmem_ld32(t_row + up_off + c * 64 + 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_swiglu(g + 8 * q, u + 8 * q, seg[4 + q]);
+    } else if (EPI == MOE_EPI_STORE) {
+      float v[32];
+      tmem_ld32(t_row + c * 64, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_bf16(v + 8 * q, 1.0f, seg[q]);
+      tmem_ld32(t_row + c * 64 + 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pack8_bf16(v + 8 * q, 1.0f, seg[4 + q]);
+    } else {
+      float v[32];
+      tmem_ld32(t_row + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        seg[q] = make_uint4(__float_as_uint(v[4 * q] * scale), __float_as_uint(v[4 * q + 1] * scale),
+                            __float_as_uint(v[4 * q + 2] * scale),
+                            __float_as_uint(v[4 * q + 3] * scale));
+    }
+    const int32_t seg_cols = EPI == MOE_EPI_WEIGHT_SCATTER ? 32 : 64;
+    uint8_t* d = (row_dst != nullptr && c * seg_cols < n_left) ? row_dst + c * 128 : nullptr;
+    warp_store_rows128(seg, d, buf, lane);
+  }
+}
+
 // The epilogue of one 128-row accumulator tile (this warp: 32 of the rows).
 //   EPI = MOE_EPI_STORE           bf16 C[row, col0 + 0..255]     (4 segments)
 //         MOE_EPI_SWIGLU          bf16 C[row, col0 + 0..127] from gate cols

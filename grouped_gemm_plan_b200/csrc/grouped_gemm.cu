@@ -383,18 +383,15 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
                             const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                             int num_sms, cudaStream_t stream);
 
-// Which kernel runs a grouped GEMM.  The CTA-pair kernel (256-row tiles) moves a
-// third fewer bytes into each SM per MMA and wins once experts hold many rows;
-// with fewer rows per expert its 256-row tiles pad more rows than the
-// single-CTA kernel's 128-row tiles and it loses.  Measured on B200: pair faster
-// at 1024 and 2048 rows per expert (Mixtral and Phi-3.5 shapes), slower at 512
-// and 256 (Qwen2 and wide M=512 shapes).  MOE_GEMM_PAIR=0/1 in the environment
-// forces one kernel (the tests run both).
+// Which kernel runs a grouped GEMM: the CTA-pair kernel (grouped_gemm_2sm.cu),
+// which moves a third fewer bytes into each SM per MMA, takes its tiles from the
+// device tile queue and pads short experts only to 128 rows, on every shape; this
+// single-CTA kernel (128-row tiles, static tile walk) when MOE_GEMM_PAIR=0 forces
+// it (comparisons; the tests run both), or on a device with a single SM.
 static bool use_pair_kernel(int64_t R, int32_t E) {
   const char* v = getenv("MOE_GEMM_PAIR");
   if (v != nullptr && v[0] == '0') return false;
-  if (v != nullptr && v[0] == '1') return true;
-  return E > 0 && R >= 1024 * static_cast<int64_t>(E);
+  return R > 0 && E > 0;
 }
 
 static int launch_grouped_gemm_1sm(const void* A, const void* B, const int32_t* offsets, int32_t E,

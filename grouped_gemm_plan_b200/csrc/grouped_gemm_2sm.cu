@@ -1,24 +1,40 @@
-// grouped_gemm_2sm.cu -- the grouped GEMM on CTA pairs: tcgen05.mma.cta_group::2
-// with a 256 x 256 tile per pair of SMs.
+// grouped_gemm_2sm.cu -- the grouped GEMM on CTA pairs (tcgen05.mma.cta_group::2)
+// fed from a device tile queue.
 //
-// Same computation and tile order as grouped_gemm.cu ("Grouped GEMM 为什么适合
-// MoE", sections "Grouped GEMM 到底解决什么问题", "1. Tiling", "2. Double-buffer
-// pipeline", "Fused GemmAdd"); the difference is how a tile is fed.  A cluster of
-// two CTAs on neighbouring SMs shares one 256-row m-tile: each CTA loads its own
-// 128 rows of A and one half (128 columns) of B, and the leader CTA issues one
-// M = 256, N = 256 MMA that reads A and B from both CTAs' shared memory and
-// writes each CTA's 128 rows of the accumulator into that CTA's TMEM.  Per SM
-// that halves the B bytes fetched for the same work (32 KB per 64 of K instead
-// of 48 KB).  A stage holds 128 of K (eight MMAs per barrier round trip, three
-// 64 KB stages), since the pair's barrier hand-offs cross SMs and cost more per
-// round trip than the single-CTA kernel's.
+// What it computes ("Grouped GEMM 为什么适合 MoE", section "Grouped GEMM 到底解决什么
+// 问题"): C_e = A_e x B_e for every expert e, A_e the row segment [offsets[e],
+// offsets[e+1]) of the expert-ordered activations, B_e = B[e]; the epilogue as in
+// grouped_gemm.cu ("Fused GemmAdd": fp32 math on the accumulator, one cast).
 //
-// Protocol (leader = cluster rank 0, peer = rank 1):
-//   full[s]    leader's barrier; the leader arrives with the byte count of both
-//              CTAs' loads; both CTAs' TMA loads complete their bytes on it
-//   empty[s]   in each CTA; the leader's MMA thread commits to both
-//   tfull[b]   in each CTA; the leader commits to both after a tile's last MMA
-//   tempty[b]  leader's barrier; one arrival per epilogue warp of both CTAs
+// Scheduling (same section: a fixed set of CTAs keeps asking which expert's which
+// tile comes next; "什么时候 Grouped GEMM 不一定赚": long tails need finer
+// splitting): the grid is one CTA pair per two SMs, persistent.  The work is one
+// list of tiles, expert by expert, and inside an expert n-tile outer, m-tile inner
+// ("1. Tiling"), so the pairs running at the same time share a B column block.
+// The leader CTA of a pair takes the next tile from an atomic ticket counter in
+// the workspace (the device tile queue) when its producer starts a tile, and hands
+// it to its own MMA and epilogue warps and to the peer CTA through a small ring in
+// shared memory.  Tile shapes:
+//   - full tiles: 256 rows x 256 accumulator columns (M = 256, N = 256), each CTA
+//     loading its 128 rows of A and its half of B;
+//   - an expert's last m-tile with at most 128 rows: M = 128 (64 rows per CTA), so
+//     a short expert pads to a multiple of 128 rows rather than 256;
+//   - when the last partial wave holds at most half as many tiles as there are
+//     pairs, its tiles are issued as two N = 128 halves each, so the final wave
+//     ends earlier.
+// The ticket counter is reset to zero by the last CTA of the grid to finish.  The
+// tile a pair computes does not change its arithmetic (no split-K, fixed K order),
+// so results are bit-identical whichever pair takes which tile.
+//
+// Pipeline (per pair): TMA loads of both CTAs complete on the leader's stage
+// barrier; the leader's single MMA thread issues eight MMAs (128 of K) per stage
+// and commits to both CTAs' barriers; two TMEM accumulators let the epilogue of
+// one tile overlap the next tile's main loop ("2. Double-buffer pipeline").
+//
+// TMEM layout of the accumulator (per CTA, 128 lanes): M = 256: lane l = row
+// 128 * rank + l, column n = output column n.  M = 128: the CTA's 64 rows appear
+// twice, lanes [0, 64) hold columns [0, 128) and lanes [64, 128) hold columns
+// [128, 256), each in TMEM columns [0, 128).
 // Peer addresses come from mapa.  No load is multicast.
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -28,7 +44,7 @@ namespace moe {
 
 namespace {
 
-constexpr int P_BM = 256;                 // rows per CTA pair
+constexpr int P_BM = 256;                 // rows of a full pair tile
 constexpr int P_BN = 256;
 constexpr int P_BK = 128;                 // K per stage: 8 MMAs per barrier round trip
 constexpr int P_STAGES = 3;
@@ -40,7 +56,15 @@ constexpr int P_B_BYTES = 2 * P_B_BOX_BYTES;    // this CTA's 128 columns
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_TMEM_COLS = 512;
 constexpr int P_DYN_SMEM = P_STAGES * P_STAGE_BYTES + 4 * EPI_STAGE_BYTES_PER_WARP + 1024;
-constexpr uint32_t P_IDESC = idesc_bf16_f32(256, P_BN, true);
+constexpr int P_RING = 8;                 // tile ring entries
+// consumers of a ring entry: leader MMA thread, 4 epilogue warps in each CTA, peer producer
+constexpr uint32_t P_RING_CONSUMERS = 1 + 4 + 4 + 1;
+
+// Tile variants in the ring
+constexpr int32_t V_WHOLE = 0;            // all 256 accumulator columns
+constexpr int32_t V_HALF0 = 1;            // accumulator columns [0, 128) of the tile
+constexpr int32_t V_HALF1 = 2;            // accumulator columns [128, 256)
+constexpr int32_t T_END = -1;
 
 struct Gemm2Args {
   const int32_t* offsets;
@@ -52,11 +76,13 @@ struct Gemm2Args {
   float* Cf;
   int64_t ldc;
   int32_t* status;
+  int32_t* queue;      // [0] ticket counter, [1] CTAs finished (both zero between launches)
   uint64_t timeout_ns;
 };
 
 struct PTile {
   int32_t e, row0, rows, ni;
+  bool m128;           // M = 128 tile (at most 128 valid rows)
 };
 
 __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, const int32_t* s_off,
@@ -75,7 +101,35 @@ __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, con
   const int32_t mi = local - c.ni * mt;
   c.row0 = s_off[e] + mi * P_BM;
   c.rows = min(P_BM, s_off[e + 1] - c.row0);
+  c.m128 = c.rows <= 128;
   return c;
+}
+
+// Ticket -> (tile, variant).  Tickets [0, T - L) are whole tiles; tickets
+// [T - L, T + L) are the last L tiles, two tickets each: its N halves, or for an
+// M = 128 tile the whole tile on the first ticket and nothing (skip, returns
+// false) on the second.
+__device__ __forceinline__ bool ticket_to_tile(int32_t ticket, int32_t T, int32_t L,
+                                               const int32_t* s_tstart, const int32_t* s_off,
+                                               int32_t E, int32_t* tile, int32_t* variant) {
+  if (ticket < T - L) {
+    *tile = ticket;
+    *variant = V_WHOLE;
+    return true;
+  }
+  const int32_t u = ticket - (T - L);
+  *tile = T - L + (u >> 1);
+  const PTile pt = decode2(*tile, s_tstart, s_off, E);
+  if (pt.m128) {
+    *variant = V_WHOLE;
+    return (u & 1) == 0;
+  }
+  *variant = (u & 1) ? V_HALF1 : V_HALF0;
+  return true;
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, int32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 }  // namespace
@@ -83,6 +137,7 @@ __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, con
 template <int EPI>
 __global__ void __launch_bounds__(P_THREADS, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmA64,
                             const __grid_constant__ CUtensorMap tmB, const Gemm2Args args) {
   extern __shared__ uint8_t p_dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[P_STAGES];
@@ -90,6 +145,10 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t ring_full[P_RING];
+  __shared__ __align__(8) uint64_t ring_empty[P_RING];
+  __shared__ int32_t s_ring_tile[P_RING];
+  __shared__ int32_t s_ring_var[P_RING];
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int32_t s_abort;
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
@@ -99,7 +158,6 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   const int32_t E = args.E;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
-  const int32_t pair = static_cast<int32_t>(blockIdx.x) >> 1;
   const int32_t npairs = static_cast<int32_t>(gridDim.x) >> 1;
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(p_dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -113,6 +171,10 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 8);  // 4 epilogue warps in each CTA of the pair
     }
+    for (int q = 0; q < P_RING; ++q) {
+      mbar_init(&ring_full[q], 1);
+      mbar_init(&ring_empty[q], P_RING_CONSUMERS);
+    }
     mbar_init(&drain_bar, 1);
     s_abort = 0;
     fence_barrier_init();
@@ -120,6 +182,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA64);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
@@ -160,49 +223,143 @@ __global__ void __launch_bounds__(P_THREADS, 1)
 
   const uint32_t tmem_base = s_tmem_base;
   const int32_t T = s_tstart[E];
+  // Tiles issued as two tickets: the last partial wave's tiles, when their halves
+  // fit one wave (a half tile costs more than half a tile, so splitting a wave that
+  // is more than half full would make the end later, not earlier).
+  const int32_t r_last = T % npairs;
+  const int32_t L = 2 * r_last <= npairs ? r_last : 0;
+  const int32_t tickets = T + L;
   const int32_t KB = (args.K + P_BK - 1) / P_BK;  // a short last k-block reads zeros
+
+  // Waits for ring entry j and returns it (tile, variant); T_END when the list is
+  // done or the wait ran out (then the abort flag is set).  Releases the entry: a
+  // local arrival in the leader CTA, a remote one from the peer.
+  auto ring_take = [&](uint32_t j, int32_t* var) -> int32_t {
+    const uint32_t slot = j % P_RING, ph = (j / P_RING) & 1u;
+    if (!mbar_wait_cluster(&ring_full[slot], ph, args.timeout_ns, &s_abort)) {
+      set_status(args.status, MOE_ERR_TIMEOUT);
+      s_abort = 1;
+      return T_END;
+    }
+    const int32_t t = s_ring_tile[slot];
+    *var = s_ring_var[slot];
+    if (leader)
+      mbar_arrive(&ring_empty[slot]);
+    else
+      mbar_arrive_cluster(peer_addr(smem_u32(&ring_empty[slot]), 0));
+    return t;
+  };
+
+  // Leader only: resolves a ticket into ring entry j (tile and variant, taking more
+  // tickets past the empty second tickets of M = 128 tail tiles) and hands it to
+  // both CTAs.  Returns false if the wait for the ring slot ran out.
+  auto ring_push = [&](uint32_t j, int32_t ticket, int32_t* t_out, int32_t* var_out) -> bool {
+    int32_t t = T_END, var = V_WHOLE;
+    for (;; ticket = atomicAdd(args.queue, 1)) {
+      if (ticket < 0 || ticket >= tickets) {
+        t = T_END;
+        break;
+      }
+      if (ticket_to_tile(ticket, T, L, s_tstart, s_off, E, &t, &var)) break;
+    }
+    // this pair's last tile is under way: the next kernel may be scheduled
+    if (t == T_END) griddep_launch_dependents();
+    const uint32_t slot = j % P_RING, ph = (j / P_RING) & 1u;
+    if (!mbar_wait_cluster(&ring_empty[slot], ph ^ 1u, args.timeout_ns, &s_abort)) {
+      set_status(args.status, MOE_ERR_TIMEOUT);
+      s_abort = 1;
+      return false;
+    }
+    s_ring_tile[slot] = t;
+    s_ring_var[slot] = var;
+    st_cluster_u32(peer_addr(smem_u32(&s_ring_tile[slot]), 1), t);
+    st_cluster_u32(peer_addr(smem_u32(&s_ring_var[slot]), 1), var);
+    mbar_arrive_cluster(peer_addr(smem_u32(&ring_full[slot]), 0));
+    mbar_arrive_cluster(peer_addr(smem_u32(&ring_full[slot]), 1));
+    *t_out = t;
+    *var_out = var;
+    return true;
+  };
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     uint32_t stage = 0, phase = 0;
     bool issued_any = false;
-    for (int32_t t = pair; t < T && !s_abort; t += npairs) {
-      // the next kernel may be scheduled once every CTA is on its last tile
-      if (t + npairs >= T) griddep_launch_dependents();
+    // The leader hands out tile j + 1 while it issues the last k-blocks of tile j:
+    // it takes the ticket four k-blocks before the end (the atomic's round trip to
+    // L2 overlaps those loads) and pushes the entry two k-blocks before the end,
+    // after that k-block's loads are issued, so neither producer waits for it at
+    // the tile boundary.
+    int32_t t = T_END, var = V_WHOLE;
+    bool pushed = true;
+    if (leader) pushed = ring_push(0, atomicAdd(args.queue, 1), &t, &var);
+    for (uint32_t j = 0; !s_abort && pushed; ++j) {
+      if (!leader) {
+        t = ring_take(j, &var);
+        if (t == T_END) griddep_launch_dependents();
+      }
+      if (t == T_END) break;
       const PTile tc = decode2(t, s_tstart, s_off, E);
-      const int32_t arow = tc.row0 + 128 * static_cast<int32_t>(rank);
+      const bool half = var != V_WHOLE;
+      const int32_t h = var == V_HALF1 ? 1 : 0;
+      // this CTA's A rows: 128 of a full tile, 64 of an M = 128 tile
+      const int32_t arow = tc.row0 + (tc.m128 ? 64 : 128) * static_cast<int32_t>(rank);
+      const uint32_t a_bytes = tc.m128 ? P_A_BYTES / 2 : P_A_BYTES;
+      const int nbox = half ? 1 : 2;  // B boxes of 64 columns this CTA loads
+      const uint32_t cta_bytes = a_bytes + static_cast<uint32_t>(nbox) * P_B_BOX_BYTES;
+      const int32_t kb_fetch = KB > 4 ? KB - 4 : 0;
+      const int32_t kb_push = KB > 2 ? KB - 2 : 0;
+      int32_t next_ticket = 0, next_t = T_END, next_var = V_WHOLE;
+      bool next_pushed = false;
       for (int32_t kb = 0; kb < KB; ++kb) {
         if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.timeout_ns, &s_abort)) {
           set_status(args.status, MOE_ERR_TIMEOUT);
           s_abort = 1;
           break;
         }
+        if (leader && kb == kb_fetch) next_ticket = atomicAdd(args.queue, 1);
         const uint32_t fb = peer_addr(smem_u32(&full_bar[stage]), 0);
         if (leader) {
           asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
                            smem_u32(&full_bar[stage])),
-                       "r"(2 * P_STAGE_BYTES)
+                       "r"(2 * cta_bytes)
                        : "memory");
         }
         uint8_t* sa = ring + stage * P_STAGE_BYTES;
         uint8_t* sb = sa + P_A_BYTES;
 #pragma unroll
         for (int c = 0; c < P_BK / 64; ++c)
-          tma2_load_2d(sa + c * P_A_BOX_BYTES, &tmA, fb, kb * P_BK + 64 * c, arow);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
+          tma2_load_2d(sa + c * P_A_BOX_BYTES, tc.m128 ? &tmA64 : &tmA, fb, kb * P_BK + 64 * c, arow);
+        for (int b = 0; b < nbox; ++b) {
           int32_t n;
-          if (EPI == MOE_EPI_SWIGLU)  // leader: gate columns, peer: up columns
-            n = (rank == 0 ? 0 : args.up_col) + tc.ni * 128 + 64 * j;
-          else
-            n = tc.ni * P_BN + 128 * static_cast<int32_t>(rank) + 64 * j;
-          tma2_load_3d(sb + j * P_B_BOX_BYTES, &tmB, fb, n, kb * P_BK, tc.e);
+          if (EPI == MOE_EPI_SWIGLU) {
+            const int32_t j0 = tc.ni * 128;
+            if (half)            // leader: gate, peer: up, 64 columns of the half
+              n = (rank == 0 ? 0 : args.up_col) + j0 + 64 * h;
+            else if (tc.m128)    // each CTA: 64 gate columns, then the same 64 up columns
+              n = (b == 0 ? 0 : args.up_col) + j0 + 64 * static_cast<int32_t>(rank);
+            else                 // leader: 128 gate columns, peer: 128 up columns
+              n = (rank == 0 ? 0 : args.up_col) + j0 + 64 * b;
+          } else {
+            n = half ? tc.ni * P_BN + 128 * h + 64 * static_cast<int32_t>(rank)
+                     : tc.ni * P_BN + 128 * static_cast<int32_t>(rank) + 64 * b;
+          }
+          tma2_load_3d(sb + b * P_B_BOX_BYTES, &tmB, fb, n, kb * P_BK, tc.e);
         }
         issued_any = true;
         if (++stage == P_STAGES) {
           stage = 0;
           phase ^= 1u;
         }
+        if (leader && kb == kb_push) {
+          next_pushed = ring_push(j + 1, next_ticket, &next_t, &next_var);
+          if (!next_pushed) break;
+        }
+      }
+      if (leader) {
+        if (!next_pushed) break;   // abort before the next entry was handed out
+        t = next_t;
+        var = next_var;
       }
     }
     if (s_abort && issued_any) {
@@ -212,9 +369,15 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer (leader)
-    uint32_t stage = 0, phase = 0, j = 0;
+    uint32_t stage = 0, phase = 0;
     bool issued_any = false;
-    for (int32_t t = pair; t < T && !s_abort; t += npairs, ++j) {
+    for (uint32_t j = 0; !s_abort; ++j) {
+      int32_t var = V_WHOLE;
+      const int32_t t = ring_take(j, &var);
+      if (t == T_END) break;
+      const PTile tc = decode2(t, s_tstart, s_off, E);
+      const uint32_t idesc = var != V_WHOLE ? idesc_bf16_f32(256, 128, true)
+                                            : idesc_bf16_f32(tc.m128 ? 128 : 256, P_BN, true);
       const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
       if (!mbar_wait_cluster(&tempty_bar[b], tph ^ 1u, args.timeout_ns, &s_abort)) {
         set_status(args.status, MOE_ERR_TIMEOUT);
@@ -236,7 +399,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         for (int kk = 0; kk < P_BK / 16; ++kk) {
           const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * P_A_BOX_BYTES + (kk & 3) * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, P_B_BOX_BYTES, 1024);
-          umma2_bf16(d_tmem, adesc, bdesc, P_IDESC, (kb | kk) != 0 ? 1u : 0u);
+          umma2_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         issued_any = true;
         const uint32_t eb = smem_u32(&empty_bar[stage]);
@@ -258,15 +421,17 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const int rr = q * 32 + lane;                          // row of this CTA's half
-    const int r = 128 * static_cast<int>(rank) + rr;        // row of the pair's tile
+    const int q = warp & 3;              // TMEM sub-partition of this warp: lanes [32q, 32q + 32)
     uint4* stage_buf = reinterpret_cast<uint4*>(ring + P_STAGES * P_STAGE_BYTES +
                                                 (warp - 2) * EPI_STAGE_BYTES_PER_WARP);
     const uint32_t te_leader0 = peer_addr(smem_u32(&tempty_bar[0]), 0);
     const uint32_t te_leader1 = peer_addr(smem_u32(&tempty_bar[1]), 0);
-    uint32_t j = 0;
-    for (int32_t t = pair; t < T && !s_abort; t += npairs, ++j) {
+    for (uint32_t j = 0; !s_abort; ++j) {
+      int32_t t = 0, var = V_WHOLE;
+      if (lane == 0) t = ring_take(j, &var);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      var = __shfl_sync(0xffffffffu, var, 0);
+      if (t == T_END) break;
       const PTile tc = decode2(t, s_tstart, s_off, E);
       const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
       int32_t okw = 1;
@@ -282,20 +447,37 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       __syncwarp();
       tc_fence_after();
       const uint32_t t_row = tmem_base + b * P_BN + (static_cast<uint32_t>(q * 32) << 16);
+      // which rows and output columns this warp's lanes hold
+      int32_t r, col0, nseg;
+      uint32_t up_off;
+      const int32_t h = var == V_HALF1 ? 1 : 0;
+      if (tc.m128) {
+        r = 64 * static_cast<int32_t>(rank) + 32 * (q & 1) + lane;
+        const int32_t nh = q >> 1;       // lanes [64, 128) hold accumulator columns [128, 256)
+        if (EPI == MOE_EPI_SWIGLU) {
+          col0 = tc.ni * 128 + 64 * nh;
+          nseg = 1;
+          up_off = 64;
+        } else {
+          col0 = tc.ni * P_BN + 128 * nh;
+          nseg = EPI == MOE_EPI_WEIGHT_SCATTER ? 4 : 2;
+          up_off = 0;
+        }
+      } else {
+        r = 128 * static_cast<int32_t>(rank) + 32 * q + lane;
+        if (EPI == MOE_EPI_SWIGLU) {
+          col0 = tc.ni * 128 + (var != V_WHOLE ? 64 * h : 0);
+          nseg = var != V_WHOLE ? 1 : 2;
+          up_off = var != V_WHOLE ? 64 : 128;
+        } else {
+          col0 = tc.ni * P_BN + (var != V_WHOLE ? 128 * h : 0);
+          nseg = (EPI == MOE_EPI_WEIGHT_SCATTER ? 8 : 4) / (var != V_WHOLE ? 2 : 1);
+          up_off = 0;
+        }
+      }
       const bool row_ok = r < tc.rows;
       const int32_t s = tc.row0 + r;
-      if (EPI == MOE_EPI_SWIGLU) {
-        const int32_t col0 = tc.ni * 128;
-        uint8_t* dst = row_ok ? reinterpret_cast<uint8_t*>(args.C + static_cast<int64_t>(s) * args.ldc + col0)
-                              : nullptr;
-        epilogue_tile<MOE_EPI_SWIGLU>(t_row, dst, args.n_out - col0, 1.0f, stage_buf, lane);
-      } else if (EPI == MOE_EPI_STORE) {
-        const int32_t col0 = tc.ni * P_BN;
-        uint8_t* dst = row_ok ? reinterpret_cast<uint8_t*>(args.C + static_cast<int64_t>(s) * args.ldc + col0)
-                              : nullptr;
-        epilogue_tile<MOE_EPI_STORE>(t_row, dst, args.n_out - col0, 1.0f, stage_buf, lane);
-      } else {
-        const int32_t col0 = tc.ni * P_BN;
+      if (EPI == MOE_EPI_WEIGHT_SCATTER) {
         float scale = 1.0f;
         uint8_t* dst = nullptr;
         if (row_ok) {
@@ -306,7 +488,12 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           else
             dst = reinterpret_cast<uint8_t*>(args.Cf + static_cast<int64_t>(dest) * args.ldc + col0);
         }
-        epilogue_tile<MOE_EPI_WEIGHT_SCATTER>(t_row, dst, args.n_out - col0, scale, stage_buf, lane);
+        epilogue_segments<MOE_EPI_WEIGHT_SCATTER>(t_row, dst, args.n_out - col0, nseg, 0, scale,
+                                                  stage_buf, lane);
+      } else {
+        uint8_t* dst = row_ok ? reinterpret_cast<uint8_t*>(args.C + static_cast<int64_t>(s) * args.ldc + col0)
+                              : nullptr;
+        epilogue_segments<EPI>(t_row, dst, args.n_out - col0, nseg, up_off, 1.0f, stage_buf, lane);
       }
       tc_fence_before();
       __syncwarp();
@@ -316,11 +503,19 @@ __global__ void __launch_bounds__(P_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // the peer no longer touches this CTA's barriers or TMEM
+  cluster_sync();  // the peer no longer touches this CTA's barriers, ring or TMEM
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc2(tmem_base, P_TMEM_COLS);
+  }
+  if (tid == 0) {
+    // the last CTA to finish leaves the queue at zero for the next launch
+    __threadfence();
+    if (atomicAdd(args.queue + 1, 1) == static_cast<int32_t>(gridDim.x) - 1) {
+      atomicExch(args.queue, 0);
+      atomicExch(args.queue + 1, 0);
+    }
   }
 }
 
@@ -337,8 +532,8 @@ static bool enc2(CUtensorMap* m, int rank, const void* base, const cuuint64_t* d
 }
 
 template <int EPI>
-static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& b,
-                             const Gemm2Args& args, cudaStream_t stream) {
+static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& a64,
+                             const CUtensorMap& b, const Gemm2Args& args, cudaStream_t stream) {
   static PerDeviceOnce once;
   const cudaError_t err = once.run([] {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>,
@@ -350,24 +545,29 @@ static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& 
   });
   if (err != cudaSuccess) return err;
   return launch_pdl(grouped_gemm_2sm_kernel<EPI>, dim3(static_cast<unsigned>(grid)), dim3(P_THREADS),
-                    P_DYN_SMEM, stream, 2, a, b, args);
+                    P_DYN_SMEM, stream, 2, a, a64, b, args);
 }
 
-// Same contract as launch_grouped_gemm (0 ok, 1 tensor map, 2 CUDA error).
+// Same contract as launch_grouped_gemm (0 ok, 1 tensor map, 2 CUDA error).  `status`
+// is the workspace's status word; the tile queue lives at status + 32 (byte 128 of
+// the workspace's 256-byte control block).
 int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets, int32_t E,
                             int64_t R, int64_t K, int64_t N, int epi, const float* w_sorted,
                             const int32_t* perm, void* C, int32_t* status, uint64_t timeout_ns,
                             int num_sms, cudaStream_t stream) {
   if (R == 0) return 0;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmA64, tmB;
   const cuuint64_t adims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(R)};
   const cuuint64_t astr[1] = {static_cast<cuuint64_t>(K) * 2};
   const cuuint32_t abox[2] = {64, 128};
+  const cuuint32_t abox64[2] = {64, 64};
   const cuuint64_t bdims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
                                static_cast<cuuint64_t>(E)};
   const cuuint64_t bstr[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(K * N) * 2};
   const cuuint32_t bbox[3] = {64, P_BK, 1};
-  if (!enc2(&tmA, 2, A, adims, astr, abox) || !enc2(&tmB, 3, B, bdims, bstr, bbox)) return 1;
+  if (!enc2(&tmA, 2, A, adims, astr, abox) || !enc2(&tmA64, 2, A, adims, astr, abox64) ||
+      !enc2(&tmB, 3, B, bdims, bstr, bbox))
+    return 1;
   Gemm2Args a;
   a.offsets = offsets;
   a.E = E;
@@ -378,6 +578,7 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
   a.C = static_cast<__nv_bfloat16*>(C);
   a.Cf = static_cast<float*>(C);
   a.status = status;
+  a.queue = status + 32;
   a.timeout_ns = timeout_ns;
   if (epi == MOE_EPI_SWIGLU) {
     a.n_out = static_cast<int32_t>(N / 2);
@@ -392,16 +593,16 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
   }
   const int64_t tiles_max = (R / P_BM + (E < R ? E : R)) * a.n_tiles_n;
   int64_t pairs = num_sms / 2;
-  if (tiles_max < pairs) pairs = tiles_max;
+  if (2 * tiles_max < pairs) pairs = 2 * tiles_max;   // the last tiles run as two halves
   if (pairs < 1) pairs = 1;
   const int grid = static_cast<int>(2 * pairs);
   cudaError_t err;
   if (epi == MOE_EPI_SWIGLU)
-    err = launch2_t<MOE_EPI_SWIGLU>(grid, tmA, tmB, a, stream);
+    err = launch2_t<MOE_EPI_SWIGLU>(grid, tmA, tmA64, tmB, a, stream);
   else if (epi == MOE_EPI_WEIGHT_SCATTER)
-    err = launch2_t<MOE_EPI_WEIGHT_SCATTER>(grid, tmA, tmB, a, stream);
+    err = launch2_t<MOE_EPI_WEIGHT_SCATTER>(grid, tmA, tmA64, tmB, a, stream);
   else
-    err = launch2_t<MOE_EPI_STORE>(grid, tmA, tmB, a, stream);
+    err = launch2_t<MOE_EPI_STORE>(grid, tmA, tmA64, tmB, a, stream);
   return err == cudaSuccess ? 0 : 2;
 }
 

@@ -95,11 +95,13 @@ typedef enum moe_op {
 int moe_abi_version(void);
 
 /* Bytes of device workspace `op` needs for this shape (always >= 256; the first
- * 256 bytes hold the device status word; the plan also keeps per-chunk expert
- * histograms there, 256 * (E + 1) int32).  The workspace must be 256-byte
- * aligned.  Its contents need no initialisation except that the status word
- * should read 0 before the first call (zero the buffer once, or call
- * moe_get_device_status once, which clears it). */
+ * 256 bytes are a control block: the device status word and the grouped GEMM's
+ * tile queue; the plan also keeps per-chunk expert histograms after it, 256 *
+ * (E + 1) int32).  The workspace must be 256-byte aligned.  Its contents need no
+ * initialisation except that the control block must read 0 before the first
+ * call (zero the buffer once, or call moe_get_device_status once, which clears
+ * it); every call leaves the tile queue at zero again.  A workspace serves one
+ * call at a time: calls that overlap on the GPU need workspaces of their own. */
 size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
 
 /*
@@ -137,6 +139,23 @@ moe_status moe_plan(const int32_t* topk_ids, const float* topk_w, int64_t M, int
                     int32_t topk, int32_t* counts, int32_t* offsets, int32_t* perm,
                     int32_t* inv_perm, float* w_sorted, void* ws, size_t ws_bytes,
                     void* stream);
+
+/*
+ * moe_route_plan -- moe_route and moe_plan in one call, the routing front end
+ * fused with the plan's first pass ([PTO] "MegaMoE 融合算子七阶段": FrontReorder
+ * directly behind the router): one kernel routes every token (as moe_route) and
+ * counts its routed rows per expert into per-chunk histograms in the workspace;
+ * a second kernel scans them into offsets and scatters the stable permutation.
+ *   logits fp32 [M, E]; out: topk_ids int32 [M, topk], topk_w fp32 [M, topk]
+ *   (exactly as moe_route writes them), counts [E], offsets [E+1], perm [R],
+ *   inv_perm [R] (may be NULL), w_sorted [R] (may be NULL): exactly as moe_plan
+ *   writes them for those ids and weights.
+ * Workspace: moe_workspace_size(MOE_OP_PLAN, ...).  topk <= min(E, 32).
+ */
+moe_status moe_route_plan(const float* logits, int64_t M, int32_t E, int32_t topk,
+                          int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv_perm, float* w_sorted, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /*
  * moe_dispatch -- permute ([PTO] Dispatch; [COMET] 3.2, layer 0 token dispatch):
@@ -339,7 +358,8 @@ moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
                              size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns the device status word of `ws` (a moe_status)
- * and clears it to MOE_OK.  Returns MOE_ERR_CUDA if the stream reports an error. */
+ * and clears the control block (status word MOE_OK, tile queue zero).  Returns
+ * MOE_ERR_CUDA if the stream reports an error. */
 moe_status moe_get_device_status(void* ws, void* stream);
 
 /* Time limit, in nanoseconds, of every bounded device-side wait (default 2 s).

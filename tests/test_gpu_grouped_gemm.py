@@ -159,3 +159,61 @@ def test_repeat_is_bitwise_deterministic(cuda_dev):
     c = _run(cuda_dev, A, Bw, off, B.EPI_WEIGHT_SCATTER, 512, w_sorted=w_sorted, perm=perm)
     d = _run(cuda_dev, A, Bw, off, B.EPI_WEIGHT_SCATTER, 512, w_sorted=w_sorted, perm=perm)
     assert torch.equal(c.view(torch.int32), d.view(torch.int32))
+
+
+@pytest.mark.parametrize("epi", [B.EPI_STORE, B.EPI_SWIGLU, B.EPI_WEIGHT_SCATTER])
+def test_many_tiles_mixed_shapes(cuda_dev, epi):
+    """More tiles than CTA pairs, experts whose last m-tile holds 1..128 rows (the
+    pair kernel's M = 128 tiles), 129..255 rows (padded 256-row tiles) and whole
+    tiles, so the tile queue hands out whole tiles first and N halves at the end;
+    one-hot A rows make every output exact."""
+    counts = [600, 129, 1000, 0, 1, 383, 255, 256, 128, 64]
+    K, N = 64, 4096
+    off = _offsets(counts)
+    R, E = int(off[-1]), len(counts)
+    sel = (3 * np.arange(R) + 1) % K
+    A = torch.zeros(R, K)
+    A[np.arange(R), sel] = 1
+    A = A.to(torch.bfloat16)
+    Bw = torch.randn(E, K, N, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16)
+    G = np.zeros((R, N), np.float64)
+    for e in range(E):
+        for s in range(off[e], off[e + 1]):
+            G[s] = Bw[e, sel[s]].double().numpy()
+    if epi == B.EPI_STORE:
+        got = _run(cuda_dev, A, Bw, off, epi, N).double().numpy()
+        assert np.array_equal(got, G), _explain(got, G)
+    elif epi == B.EPI_SWIGLU:
+        got = _run(cuda_dev, A, Bw, off, epi, N // 2)
+        check_stage(got, oracle.swiglu(G), "swiglu, many tiles")
+    else:
+        rng = np.random.default_rng(9)
+        perm = rng.permutation(R).astype(np.int32)
+        w_sorted = np.exp2(rng.integers(-3, 3, R)).astype(np.float32)   # exact scaling
+        got = _run(cuda_dev, A, Bw, off, epi, N, w_sorted=w_sorted, perm=perm).double().numpy()
+        ref = np.zeros_like(G)
+        ref[perm] = w_sorted[:, None].astype(np.float64) * G
+        assert np.array_equal(got, ref), _explain(got, ref)
+
+
+def test_workspace_reused_back_to_back(cuda_dev):
+    """Consecutive launches on one workspace (the layer's GEMM1 then GEMM2 pattern):
+    each launch leaves the tile queue in the control block at zero for the next, and
+    the results equal those of launches on fresh workspaces bit for bit."""
+    off, A, Bw = _rand_case([300, 20, 900, 5], 256, 512, 12)
+    R, E = int(off[-1]), len(off) - 1
+    ws = B.alloc_workspace(B.OP_GROUPED_GEMM, R, 0, 0, E, 1, cuda_dev)
+    A_d, B_d, off_d = A.to(cuda_dev), Bw.to(cuda_dev), torch.from_numpy(off).to(cuda_dev)
+    outs = []
+    for epi, n_out in [(B.EPI_SWIGLU, 256), (B.EPI_STORE, 512), (B.EPI_SWIGLU, 256),
+                       (B.EPI_STORE, 512)]:
+        C = torch.zeros(R, n_out, dtype=torch.bfloat16, device=cuda_dev)
+        B.moe_grouped_gemm(A_d, B_d, off_d, epi, C, ws)
+        outs.append(C)
+    torch.cuda.synchronize()
+    assert int(ws[128:136].view(torch.int32).abs().sum().item()) == 0, "tile queue not reset"
+    assert B.moe_get_device_status(ws) == B.MOE_OK
+    fresh_swiglu = _run(cuda_dev, A, Bw, off, B.EPI_SWIGLU, 256)
+    fresh_store = _run(cuda_dev, A, Bw, off, B.EPI_STORE, 512)
+    for i, ref in enumerate([fresh_swiglu, fresh_store, fresh_swiglu, fresh_store]):
+        assert torch.equal(outs[i].cpu().view(torch.int16), ref.view(torch.int16)), i

@@ -66,3 +66,45 @@ def test_routed_layer(cuda_dev):
     assert np.array_equal(ids.cpu().numpy(), rid)
     ref = oracle.moe_ffn(x, W1, W2, rid, rw.astype(np.float32))
     check_close(out, ref, "routed layer")
+
+
+@pytest.mark.parametrize("M,E,topk", [(0, 8, 2), (1, 1, 1), (300, 8, 2), (4096, 8, 2),
+                                      (8192, 64, 4), (1000, 16, 3), (77, 16, 8), (513, 1024, 8),
+                                      (16384, 16, 2), (20, 33, 32)])
+def test_route_plan_matches_oracle(cuda_dev, M, E, topk):
+    """moe_route_plan: ids/weights exactly as moe_route writes them (ids bit-exact vs
+    the oracle router, weights within 1e-6), and the plan of those ids bit-exact vs
+    the oracle plan (counts, offsets, perm, inv, w_sorted) -- also for a topk that
+    does not divide the plan's chunk size."""
+    dev = cuda_dev
+    rng = np.random.default_rng(M * 11 + E)
+    logits_np = rng.standard_normal((M, E)).astype(np.float32)
+    logits = torch.from_numpy(logits_np).to(dev)
+    R = M * topk
+    ids = torch.full((M, topk), -9, dtype=torch.int32, device=dev)
+    w = torch.full((M, topk), -9.0, dtype=torch.float32, device=dev)
+    counts = torch.full((E,), -1, dtype=torch.int32, device=dev)
+    offsets = torch.full((E + 1,), -1, dtype=torch.int32, device=dev)
+    perm = torch.full((max(R, 1),), -1, dtype=torch.int32, device=dev)
+    inv = torch.full((max(R, 1),), -1, dtype=torch.int32, device=dev)
+    ws_ = torch.full((max(R, 1),), -1.0, dtype=torch.float32, device=dev)
+    ws = B.alloc_workspace(B.OP_PLAN, M, 0, 0, E, topk, dev)
+    B.moe_route_plan(logits, topk, ids, w, counts, offsets, perm[:R], inv[:R], ws_[:R], ws)
+    assert B.moe_get_device_status(ws) == B.MOE_OK
+    assert counts.cpu().tolist() == [0] * E if M == 0 else True
+    if M == 0:
+        assert offsets.cpu().tolist() == [0] * (E + 1)
+        return
+    rid, rw = oracle.route(logits_np, topk)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=0, atol=1e-6)
+    # the same ids and weights as the separate router call, bit for bit
+    ids2, w2 = _route_gpu(dev, logits_np, topk)
+    assert np.array_equal(ids.cpu().numpy(), ids2)
+    assert np.array_equal(w.cpu().numpy().view(np.int32), w2.view(np.int32))
+    rc, ro, rp, ri, rws = oracle.plan(rid, w.cpu().numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(perm[:R].cpu().numpy(), rp)
+    assert np.array_equal(inv[:R].cpu().numpy(), ri)
+    assert np.array_equal(ws_[:R].cpu().numpy(), rws)
