@@ -66,6 +66,13 @@ constexpr int32_t V_HALF0 = 1;            // accumulator columns [0, 128) of the
 constexpr int32_t V_HALF1 = 2;            // accumulator columns [128, 256)
 constexpr int32_t T_END = -1;
 
+// m-tiles per raster group of the down projection (0: the whole expert): a group's
+// activation rows stay in L2 while all of its n-tiles run ("3. L2 cache conflict
+// 缓解").  Measured on B200: GEMM2 on the Phi-3.5 shape 0.835 -> 0.844 of the bf16
+// peak; L2 eviction-priority hints on the loads (activations kept, weights evicted
+// first) made both GEMMs 1-3 % slower and are not used.
+constexpr int32_t kGroupM2 = 8;
+
 struct Gemm2Args {
   const int32_t* offsets;
   int32_t E, R, K;
@@ -85,8 +92,11 @@ struct PTile {
   bool m128;           // M = 128 tile (at most 128 valid rows)
 };
 
+// Tile t -> (expert, rows, n-tile).  Inside an expert the tiles run in groups of
+// group_m m-tiles (0: one group, the whole expert); inside a group n-tile outer,
+// m-tile inner.
 __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, const int32_t* s_off,
-                                         int32_t E) {
+                                         int32_t E, int32_t n_tiles_n, int32_t group_m) {
   int32_t lo = 0, hi = E;
   while (hi - lo > 1) {
     const int32_t mid = (lo + hi) >> 1;
@@ -94,11 +104,15 @@ __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, con
   }
   const int32_t e = lo;
   const int32_t mt = (s_off[e + 1] - s_off[e] + P_BM - 1) / P_BM;
-  const int32_t local = t - s_tstart[e];
+  int32_t local = t - s_tstart[e];
+  const int32_t gm = (group_m > 0 && group_m < mt) ? group_m : mt;
+  const int32_t g = local / (gm * n_tiles_n);
+  local -= g * gm * n_tiles_n;
+  const int32_t g_rows = min(gm, mt - g * gm);  // m-tiles in this group
   PTile c;
   c.e = e;
-  c.ni = local / mt;
-  const int32_t mi = local - c.ni * mt;
+  c.ni = local / g_rows;
+  const int32_t mi = g * gm + (local - c.ni * g_rows);
   c.row0 = s_off[e] + mi * P_BM;
   c.rows = min(P_BM, s_off[e + 1] - c.row0);
   c.m128 = c.rows <= 128;
@@ -111,7 +125,8 @@ __device__ __forceinline__ PTile decode2(int32_t t, const int32_t* s_tstart, con
 // false) on the second.
 __device__ __forceinline__ bool ticket_to_tile(int32_t ticket, int32_t T, int32_t L,
                                                const int32_t* s_tstart, const int32_t* s_off,
-                                               int32_t E, int32_t* tile, int32_t* variant) {
+                                               int32_t E, int32_t n_tiles_n, int32_t group_m,
+                                               int32_t* tile, int32_t* variant) {
   if (ticket < T - L) {
     *tile = ticket;
     *variant = V_WHOLE;
@@ -119,7 +134,7 @@ __device__ __forceinline__ bool ticket_to_tile(int32_t ticket, int32_t T, int32_
   }
   const int32_t u = ticket - (T - L);
   *tile = T - L + (u >> 1);
-  const PTile pt = decode2(*tile, s_tstart, s_off, E);
+  const PTile pt = decode2(*tile, s_tstart, s_off, E, n_tiles_n, group_m);
   if (pt.m128) {
     *variant = V_WHOLE;
     return (u & 1) == 0;
@@ -230,6 +245,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   const int32_t L = 2 * r_last <= npairs ? r_last : 0;
   const int32_t tickets = T + L;
   const int32_t KB = (args.K + P_BK - 1) / P_BK;  // a short last k-block reads zeros
+  const int32_t group_m = EPI == MOE_EPI_WEIGHT_SCATTER ? kGroupM2 : 0;
 
   // Waits for ring entry j and returns it (tile, variant); T_END when the list is
   // done or the wait ran out (then the abort flag is set).  Releases the entry: a
@@ -260,7 +276,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         t = T_END;
         break;
       }
-      if (ticket_to_tile(ticket, T, L, s_tstart, s_off, E, &t, &var)) break;
+      if (ticket_to_tile(ticket, T, L, s_tstart, s_off, E, args.n_tiles_n, group_m, &t, &var)) break;
     }
     // this pair's last tile is under way: the next kernel may be scheduled
     if (t == T_END) griddep_launch_dependents();
@@ -299,7 +315,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         if (t == T_END) griddep_launch_dependents();
       }
       if (t == T_END) break;
-      const PTile tc = decode2(t, s_tstart, s_off, E);
+      const PTile tc = decode2(t, s_tstart, s_off, E, args.n_tiles_n, group_m);
       const bool half = var != V_WHOLE;
       const int32_t h = var == V_HALF1 ? 1 : 0;
       // this CTA's A rows: 128 of a full tile, 64 of an M = 128 tile
@@ -375,7 +391,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       int32_t var = V_WHOLE;
       const int32_t t = ring_take(j, &var);
       if (t == T_END) break;
-      const PTile tc = decode2(t, s_tstart, s_off, E);
+      const PTile tc = decode2(t, s_tstart, s_off, E, args.n_tiles_n, group_m);
       const uint32_t idesc = var != V_WHOLE ? idesc_bf16_f32(256, 128, true)
                                             : idesc_bf16_f32(tc.m128 ? 128 : 256, P_BN, true);
       const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
@@ -432,7 +448,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       t = __shfl_sync(0xffffffffu, t, 0);
       var = __shfl_sync(0xffffffffu, var, 0);
       if (t == T_END) break;
-      const PTile tc = decode2(t, s_tstart, s_off, E);
+      const PTile tc = decode2(t, s_tstart, s_off, E, args.n_tiles_n, group_m);
       const uint32_t b = j & 1u, tph = (j >> 1) & 1u;
       int32_t okw = 1;
       if (lane == 0) okw = mbar_wait_bounded(&tfull_bar[b], tph, args.timeout_ns, &s_abort) ? 1 : 0;
