@@ -48,7 +48,7 @@ SIDE_DEFAULT = "tiny,mixtral,qwen2,wide16,wide128,wide512,wide2048"
 L2_NOTE = "GPU arm: L2 flushed (256 MiB write) before every timed step"
 # columns of one per-workload record
 SIDE_COLS = ["ms", "tok_s", "e2e_tok_s", "gemm1_frac", "gemm2_frac", "disp_GBs", "comb_GBs",
-             "fp8_ms", "fp8_gemm2_frac", "pair"]
+             "fp8_ms", "fp8_gemm2_frac", "route_plan_us", "pair"]
 
 
 def parse_args(argv=None):
@@ -677,6 +677,7 @@ def side_record(name, args, dev, flush, world, barrier, D, pk):
         stages = run.stage_loop(args.side_steps, barrier)
     e2e, _, _ = run.e2e_ms(args.side_steps, barrier)
     fp8 = run.fp8_leg(args.side_steps, args.side_warmup)
+    router = run.router_us()
     total, e2e = D.max_over_ranks([sum(step_ms), e2e], dev)
     rates = run.rates(stages, pk["bf16_tflops"], pk["hbm_gbs"])
     rec = [_r(total / args.side_steps), _r(D.whole_job_rate(wl.M * args.side_steps, world, total / 1e3)),
@@ -684,6 +685,7 @@ def side_record(name, args, dev, flush, world, barrier, D, pk):
            _r(rates["gemm1_frac"], 3), _r(rates["gemm2_frac"], 3), _r(rates["dispatch_gbs"]),
            _r(rates["combine_gbs"]), _r(fp8["ms_per_step"]),
            _r(fp8["gemm2_e4m3_tflops"] / (2.0 * pk["bf16_tflops"]), 3),
+           _r(router["route_plan_fused_us"], 3),
            1 if gemm_uses_pair(wl.R, wl.E) else 0]
     run.free()
     return rec
