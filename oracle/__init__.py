@@ -52,6 +52,13 @@ def configure(lib):
     lib.oracle_bruteforce_tokens.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P]
     lib.oracle_bruteforce_tokens.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_mx_exponent.argtypes = [ctypes.c_double]
+    lib.oracle_mx_exponent.restype = ctypes.c_int
+    lib.oracle_mx_quantize_rows.argtypes = [P, i64, i64, P, P]
+    lib.oracle_mx_quantize_cols.argtypes = [P, i32, i64, i64, P, P]
+    lib.oracle_grouped_gemm_mx.argtypes = [P, P, P, P, P, i32, i64, i64, P]
+    lib.oracle_moe_ffn_mx.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P]
+    lib.oracle_moe_ffn_mx.restype = ctypes.c_int
     lib.oracle_gemm_add.argtypes = [P, P, ctypes.c_double, ctypes.c_double, i64, P]
     lib.oracle_route.argtypes = [P, i64, i32, i32, P, P]
     lib.oracle_route.restype = ctypes.c_int
@@ -309,4 +316,68 @@ def moe_ffn_fp8(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
                                     topk, _p(out))
     if st != OK:
         raise ValueError(f"oracle_moe_ffn_fp8 status {st}")
+    return out
+
+
+# ------------------------------------------------------------------ MX (block-scaled) FP8
+
+def mx_exponent(amax: float) -> int:
+    """Smallest e with amax <= 448 * 2^e (clamped to [-127, 127]; -127 for 0)."""
+    return int(_load().oracle_mx_exponent(float(amax)))
+
+
+def mx_quantize_rows(A) -> tuple[np.ndarray, np.ndarray]:
+    """Rows of A [R, K] (fp64 values, or a bf16 tensor) in blocks of 32 along K ->
+    (codes uint8 [R, K], scale exponent codes uint8 [R, K/32], value = 2^(code-127))."""
+    if isinstance(A, np.ndarray) and A.dtype == np.float64:
+        a = np.ascontiguousarray(A)
+    else:
+        import torch
+        a = np.ascontiguousarray(torch.as_tensor(A).double().numpy())
+    R, K = a.shape
+    q = np.empty((R, K), np.uint8)
+    sf = np.empty((R, K // 32), np.uint8)
+    _load().oracle_mx_quantize_rows(_p(a), R, K, _p(q), _p(sf))
+    return q, sf
+
+
+def mx_quantize_cols(B) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 B [E, K, N] per output column in blocks of 32 along K -> (codes uint8
+    [E, N, K] with K contiguous, scale exponent codes uint8 [E, N, K/32])."""
+    b = _u16(B)
+    E, K, N = b.shape
+    q = np.empty((E, N, K), np.uint8)
+    sf = np.empty((E, N, K // 32), np.uint8)
+    _load().oracle_mx_quantize_cols(_p(b), E, K, N, _p(q), _p(sf))
+    return q, sf
+
+
+def grouped_gemm_mx(Aq, a_sf, BqT, b_sf, offsets) -> np.ndarray:
+    """fp64 C [R, N] = sum over 32-blocks b of 2^(a_sf-127) 2^(b_sf-127) (Aq . BqT)_b."""
+    Aq = np.ascontiguousarray(Aq, np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, np.uint8)
+    BqT = np.ascontiguousarray(BqT, np.uint8)
+    b_sf = np.ascontiguousarray(b_sf, np.uint8)
+    offsets = np.ascontiguousarray(offsets, np.int32)
+    R, K = Aq.shape
+    E, N, _ = BqT.shape
+    C = np.zeros((R, N), np.float64)
+    _load().oracle_grouped_gemm_mx(_p(Aq), _p(a_sf), _p(BqT), _p(b_sf), _p(offsets), E, K, N,
+                                   _p(C))
+    return C
+
+
+def moe_ffn_mx(x, W1, W2, ids: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The layer with a block-scaled (MX) E4M3 down projection, fp64 [M, H]."""
+    xu, w1u, w2u = _u16(x), _u16(W1), _u16(W2)
+    M, H = xu.shape
+    E, _, F2 = w1u.shape
+    ids = np.ascontiguousarray(ids, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    topk = ids.shape[1]
+    out = np.zeros((M, H), np.float64)
+    st = _load().oracle_moe_ffn_mx(_p(xu), _p(w1u), _p(w2u), _p(ids), _p(w), M, H, F2 // 2, E,
+                                   topk, _p(out))
+    if st != OK:
+        raise ValueError(f"oracle_moe_ffn_mx status {st}")
     return out

@@ -46,6 +46,10 @@
  *   fp8 GEMM        numpy float64 matmul of the decoded operands
  *   fp8 layer       E=1,topk=1 equals torch's dense chain with the same
  *                   quantisation; within the e4m3 error bound of the exact layer
+ *   mx fp8          the exponent rule vs a brute-force search; the quantisers vs
+ *                   torch's e4m3 conversion of the exactly scaled values; the MX
+ *                   GEMM vs numpy block by block; the MX layer within the E4M3
+ *                   error bound of the exact layer
  *   gemm add        beta = 0 and alpha = 0 reduce to the layer and to the added
  *                   tensor exactly; (out - add) of the residual form equals the
  *                   layer; linear in alpha and beta
@@ -423,12 +427,12 @@ double oracle_e4m3_decode(uint8_t c)
  * beyond 448 saturate to 448 (the conversion the quantiser uses); NaN -> 0x7F.
  * Every step is exact in fp64: |v| is a float, the grid spacing a power of two.
  */
-uint8_t oracle_e4m3_encode(float v)
+static uint8_t e4m3_encode_d(double v)
 {
     if (isnan(v))
         return 0x7F;
     uint8_t sign = signbit(v) ? 0x80 : 0;
-    double a = fabs((double)v);
+    double a = fabs(v);
     /* spacing of the grid around a: 2^(e-3) in binade [2^e, 2^(e+1)), e >= -6;
        the subnormal range [0, 2^-6) has spacing 2^-9 */
     int e = -6;
@@ -455,6 +459,8 @@ uint8_t oracle_e4m3_encode(float v)
     int m = (int)((f * 2.0 - 1.0) * 8.0);
     return sign | (uint8_t)(be << 3) | (uint8_t)m;
 }
+
+uint8_t oracle_e4m3_encode(float v) { return e4m3_encode_d((double)v); }
 
 /*
  * Per-row scaled quantisation of a bf16 matrix A [R, K] (the SwiGLU output h):
@@ -531,6 +537,125 @@ void oracle_grouped_gemm_e4m3(const uint8_t *Aq, const float *a_scale, const uin
                 for (int64_t k = 0; k < K; k++)
                     acc += lut[a[k]] * lut[b[k]];
                 C[s * N + n] = (double)a_scale[s] * (double)b_scale[(int64_t)e * N + n] * acc;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------- MX (block-scaled) FP8 */
+
+/*
+ * Microscaled E4M3: elements in blocks of 32 consecutive values along the
+ * contraction dimension share one power-of-two scale 2^e, stored as the 8-bit
+ * exponent code e + 127 (E8M0: code 0 is 2^-127, 254 is 2^127, 255 unused).
+ * The reading taken here (the pages only say that SwiGLU quantises what it
+ * consumes): e is the smallest integer with amax <= 448 * 2^e, amax the block's
+ * largest magnitude, so no element of the block saturates; e = -127 for an
+ * all-zero block, clamped to [-127, 127].  q = nearest E4M3 to v * 2^-e (the
+ * scaling is exact, one rounding).
+ */
+int oracle_mx_exponent(double amax)
+{
+    if (!(amax > 0.0))
+        return -127;
+    int ex;
+    frexp(amax, &ex); /* amax in [2^(ex-1), 2^ex) */
+    /* 448 * 2^(ex-9) = 1.75 * 2^(ex-1) is the smallest candidate (448 * 2^(ex-10) < 2^(ex-1)) */
+    int e = ex - 9;
+    if (amax > ldexp(448.0, e))
+        e += 1;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return e;
+}
+
+/*
+ * Rows of A [R, K] (given values, e.g. the SwiGLU output h) quantised in blocks of
+ * 32 along K: sf[r, b] = e + 127 of block b, q[r, k] = e4m3(A[r, k] * 2^-e).
+ * K is a multiple of 32.
+ */
+void oracle_mx_quantize_rows(const double *A, int64_t R, int64_t K, uint8_t *q, uint8_t *sf)
+{
+    int64_t nb = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t b = 0; b < nb; b++) {
+            const double *v = A + r * K + b * 32;
+            double amax = 0.0;
+            for (int k = 0; k < 32; k++)
+                if (fabs(v[k]) > amax)
+                    amax = fabs(v[k]);
+            int e = oracle_mx_exponent(amax);
+            sf[r * nb + b] = (uint8_t)(e + 127);
+            for (int k = 0; k < 32; k++)
+                q[r * K + b * 32 + k] = e4m3_encode_d(ldexp(v[k], -e));
+        }
+    }
+}
+
+/*
+ * Weights B [E, K, N] (bf16, row-major, N contiguous) quantised per output column
+ * in blocks of 32 along K, written transposed (K contiguous):
+ *   sf[e, n, b] = e + 127 of the block B[e, 32b .. 32b+31, n]
+ *   qT[e, n, k] = e4m3(B[e, k, n] * 2^-e)
+ */
+void oracle_mx_quantize_cols(const uint16_t *B, int32_t E, int64_t K, int64_t N, uint8_t *qT,
+                             uint8_t *sf)
+{
+    int64_t nb = K / 32;
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *Be = B + (int64_t)e * K * N;
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; n++) {
+            for (int64_t b = 0; b < nb; b++) {
+                double amax = 0.0;
+                for (int k = 0; k < 32; k++) {
+                    double v = fabs(bf16_widen(Be[(b * 32 + k) * N + n]));
+                    if (v > amax)
+                        amax = v;
+                }
+                int ex = oracle_mx_exponent(amax);
+                sf[((int64_t)e * N + n) * nb + b] = (uint8_t)(ex + 127);
+                for (int k = 0; k < 32; k++)
+                    qT[((int64_t)e * N + n) * K + b * 32 + k] =
+                        e4m3_encode_d(ldexp(bf16_widen(Be[(b * 32 + k) * N + n]), -ex));
+            }
+        }
+    }
+}
+
+/*
+ * Grouped GEMM on block-scaled operands, exact in fp64:
+ *   C[s, n] = sum_b 2^(a_sf[s, b] - 127) * 2^(b_sf[e, n, b] - 127)
+ *                   * sum_{k in block b} decode(Aq[s, k]) * decode(BqT[e, n, k])
+ * for the rows s of expert e.  Aq [R, K], a_sf [R, K/32], BqT [E, N, K],
+ * b_sf [E, N, K/32].
+ */
+void oracle_grouped_gemm_mx(const uint8_t *Aq, const uint8_t *a_sf, const uint8_t *BqT,
+                            const uint8_t *b_sf, const int32_t *offsets, int32_t E, int64_t K,
+                            int64_t N, double *C)
+{
+    double lut[256];
+    for (int c = 0; c < 256; c++)
+        lut[c] = oracle_e4m3_decode((uint8_t)c);
+    int64_t nb = K / 32;
+    for (int32_t e = 0; e < E; e++) {
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t s = offsets[e]; s < offsets[e + 1]; s++) {
+            for (int64_t n = 0; n < N; n++) {
+                const uint8_t *a = Aq + s * K;
+                const uint8_t *bq = BqT + ((int64_t)e * N + n) * K;
+                double acc = 0.0;
+                for (int64_t b = 0; b < nb; b++) {
+                    double part = 0.0;
+                    for (int k = 0; k < 32; k++)
+                        part += lut[a[b * 32 + k]] * lut[bq[b * 32 + k]];
+                    acc += ldexp(part, (int)a_sf[s * nb + b] - 127 +
+                                           (int)b_sf[((int64_t)e * N + n) * nb + b] - 127);
+                }
+                C[s * N + n] = acc;
             }
         }
     }
@@ -629,6 +754,78 @@ done:
     free(hs);
     free(wq);
     free(ws);
+    free(yp);
+    return st;
+}
+
+/*
+ * The layer with a block-scaled (MX) E4M3 down projection, stage by stage:
+ *   plan -> dispatch -> per expert GEMM1 and SwiGLU in fp64 -> h quantised in
+ *   blocks of 32 columns (oracle_mx_quantize_rows on the fp64 values: the SwiGLU
+ *   output feeds the quantiser directly, no bf16 rounding between) -> GEMM2 on the
+ *   block-scaled operands (W2 quantised per output column in blocks of 32 rows of
+ *   F) -> weighted combine.  out fp64 [M, H].
+ */
+int oracle_moe_ffn_mx(const uint16_t *x, const uint16_t *W1, const uint16_t *W2,
+                      const int32_t *ids, const float *w, int64_t M, int64_t H, int64_t F,
+                      int32_t E, int32_t topk, double *out)
+{
+    int64_t R = M * (int64_t)topk;
+    int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t *perm = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R ? R : 1));
+    uint16_t *xp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(R ? R * H : 1));
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(R ? R * F : 1));
+    uint8_t *hq = (uint8_t *)malloc((size_t)(R ? R * F : 1));
+    uint8_t *hsf = (uint8_t *)malloc((size_t)(R ? R * (F / 32) : 1));
+    uint8_t *wq = (uint8_t *)malloc((size_t)(E * H * F));
+    uint8_t *wsf = (uint8_t *)malloc((size_t)(E * H * (F / 32)));
+    double *yp = (double *)malloc(sizeof(double) * (size_t)(R ? R * H : 1));
+    int st = ORACLE_ERR_ARG;
+    if (F % 32 != 0 || !counts || !offsets || !perm || !inv || !xp || !hd || !hq || !hsf || !wq ||
+        !wsf || !yp)
+        goto done;
+    st = oracle_plan(ids, w, M, E, topk, counts, offsets, perm, inv, NULL);
+    if (st != ORACLE_OK)
+        goto done;
+    oracle_dispatch(x, perm, M, H, topk, xp);
+    for (int32_t e = 0; e < E; e++) {
+        const uint16_t *W1e = W1 + (int64_t)e * H * 2 * F;
+#pragma omp parallel
+        {
+            double *g = (double *)malloc(sizeof(double) * (size_t)(2 * F));
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t s = offsets[e]; s < offsets[e + 1]; s++) {
+                for (int64_t j = 0; j < 2 * F; j++)
+                    g[j] = 0.0;
+                for (int64_t h = 0; h < H; h++) {
+                    double xv = bf16_widen(xp[s * H + h]);
+                    const uint16_t *wrow = W1e + h * 2 * F;
+                    for (int64_t j = 0; j < 2 * F; j++)
+                        g[j] += xv * bf16_widen(wrow[j]);
+                }
+                for (int64_t j = 0; j < F; j++)
+                    hd[s * F + j] = silu(g[j]) * g[F + j];
+            }
+            free(g);
+        }
+    }
+    oracle_mx_quantize_rows(hd, R, F, hq, hsf);
+    oracle_mx_quantize_cols(W2, E, F, H, wq, wsf);
+    oracle_grouped_gemm_mx(hq, hsf, wq, wsf, offsets, E, F, H, yp);
+    oracle_combine(yp, inv, w, M, H, topk, out);
+done:
+    free(counts);
+    free(offsets);
+    free(perm);
+    free(inv);
+    free(xp);
+    free(hd);
+    free(hq);
+    free(hsf);
+    free(wq);
+    free(wsf);
     free(yp);
     return st;
 }

@@ -48,6 +48,10 @@ MUTANTS = {
                                     "y[i] = beta * acc[i] + alpha * bf16_widen(add[i]);"),
     "gemm_add_drops_add": ("y[i] = alpha * acc[i] + beta * bf16_widen(add[i]);",
                            "y[i] = alpha * acc[i];"),
+    "mx_exponent_never_rounds_up": ("    if (amax > ldexp(448.0, e))\n        e += 1;", "    if (amax > ldexp(448.0, e + 1))\n        e += 1;"),
+    "mx_gemm_drops_b_scale": ("(int)b_sf[((int64_t)e * N + n) * nb + b] - 127);", "0);"),
+    "mx_rows_scale_not_applied": ("q[r * K + b * 32 + k] = e4m3_encode_d(ldexp(v[k], -e));",
+                                  "q[r * K + b * 32 + k] = e4m3_encode_d(v[k]);"),
     "fp8_gemm_drops_b_scale": ("C[s * N + n] = (double)a_scale[s] * (double)b_scale[(int64_t)e * N + n] * acc;",
                                "C[s * N + n] = (double)a_scale[s] * acc;"),
 }
@@ -59,7 +63,14 @@ CHILD = textwrap.dedent("""
     oracle._lib = oracle.configure(ctypes.CDLL({lib!r}))
     import test_oracle_pins as pins
     import test_oracle_fp8_pins as fp8
+    import test_oracle_mx_pins as mx
     calls = [
+        mx.test_exponent_is_the_smallest_that_fits,
+        mx.test_row_quantiser_matches_torch_e4m3,
+        mx.test_column_quantiser_matches_torch_and_round_trip,
+        mx.test_mx_gemm_matches_numpy_block_sums,
+        lambda: mx.test_mx_layer_within_e4m3_bound_of_the_exact_layer(40, 64, 96, 4, 2),
+        mx.test_mx_layer_dense_special_case,
         fp8.test_decode_every_code_matches_torch,
         fp8.test_encode_matches_torch_and_brute_force,
         fp8.test_encode_saturates,
