@@ -48,7 +48,7 @@ SIDE_DEFAULT = "tiny,mixtral,qwen2,wide16,wide128,wide512,wide2048"
 L2_NOTE = "GPU arm: L2 flushed (256 MiB write) before every timed step"
 # columns of one per-workload record
 SIDE_COLS = ["ms", "tok_s", "e2e_tok_s", "gemm1_frac", "gemm2_frac", "disp_GBs", "comb_GBs",
-             "fp8_ms", "fp8_gemm2_frac", "route_plan_us", "pair"]
+             "fp8_ms", "fp8_gemm2_frac", "mx_ms", "mx_gemm2_frac", "route_plan_us", "pair"]
 
 
 def parse_args(argv=None):
@@ -569,6 +569,50 @@ class LayerRun:
                 "gemm2_e4m3_tflops": 2.0 * R * H * F / (g8_ms / 1e3) / 1e12,
                 "rel_diff_vs_bf16_layer": rel}
 
+    def mx_leg(self, steps, warmup):
+        """The layer with the block-scaled E4M3 (MX) down projection, h quantised in
+        GEMM1's epilogue: W2 quantised once (offline, not timed), then K layer steps
+        timed like the bf16 ones, and K more with the library's stage events between
+        the launches for the per-GEMM times."""
+        torch, B, wl, dev = self.torch, self.B, self.wl, self.dev
+        M, H, F, E, topk, R = wl.M, wl.H, wl.F, wl.E, wl.topk, wl.R
+        W2q = torch.empty((E, H, F), dtype=torch.uint8, device=dev)
+        w2sf = torch.empty((E, H, F // 32), dtype=torch.uint8, device=dev)
+        B.moe_quantize_weights_mx(self.W2, W2q, w2sf)
+        wsx = B.alloc_workspace(B.OP_FFN_MX, M, H, F, E, topk, dev)
+        outx = torch.empty_like(self.out)
+
+        def mx_step():
+            B.moe_ffn_fused_mx(self.x, self.W1, W2q, w2sf, self.ids, self.tw, outx, self.counts,
+                               self.offsets, self.perm, wsx)
+        for _ in range(warmup):
+            self.flush.fill_(1)
+            mx_step()
+        ev = self.events(steps)
+        for i in range(steps):
+            self.flush.fill_(1)
+            ev[i][0].record(self.stream)
+            mx_step()
+            ev[i][1].record(self.stream)
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        for i in range(steps):
+            self.flush.fill_(1)
+            B.moe_set_stage_events(tev[i])
+            mx_step()
+        B.moe_set_stage_events(None)
+        torch.cuda.synchronize()
+        self.check_status(wsx, "in the MX layer")
+        mx_ms = _mean_ms(ev)
+        stages = {n: statistics.mean(tev[i][j].elapsed_time(tev[i][j + 1]) for i in range(steps))
+                  for j, n in enumerate(self.STAGES)}
+        of, ob = outx.float(), self.out.float()
+        rel = float(torch.linalg.norm(of - ob) / torch.linalg.norm(ob))
+        del W2q, w2sf, wsx, outx
+        return {"ms_per_step": mx_ms, "stage_ms": stages,
+                "gemm1_mx_tflops": 4.0 * R * H * F / (stages["gemm1_swiglu"] / 1e3) / 1e12,
+                "gemm2_mx_tflops": 2.0 * R * H * F / (stages["gemm2_scatter"] / 1e3) / 1e12,
+                "rel_diff_vs_bf16_layer": rel}
+
     def e2e_ms(self, steps, barrier):
         """End to end through the public call: every step's inputs are copied in from
         pinned host memory and its result copied back.  As in a serving loop, step
@@ -677,6 +721,7 @@ def side_record(name, args, dev, flush, world, barrier, D, pk):
         stages = run.stage_loop(args.side_steps, barrier)
     e2e, _, _ = run.e2e_ms(args.side_steps, barrier)
     fp8 = run.fp8_leg(args.side_steps, args.side_warmup)
+    mx = run.mx_leg(args.side_steps, args.side_warmup)
     router = run.router_us()
     total, e2e = D.max_over_ranks([sum(step_ms), e2e], dev)
     rates = run.rates(stages, pk["bf16_tflops"], pk["hbm_gbs"])
@@ -685,6 +730,7 @@ def side_record(name, args, dev, flush, world, barrier, D, pk):
            _r(rates["gemm1_frac"], 3), _r(rates["gemm2_frac"], 3), _r(rates["dispatch_gbs"]),
            _r(rates["combine_gbs"]), _r(fp8["ms_per_step"]),
            _r(fp8["gemm2_e4m3_tflops"] / (2.0 * pk["bf16_tflops"]), 3),
+           _r(mx["ms_per_step"]), _r(mx["gemm2_mx_tflops"] / (2.0 * pk["bf16_tflops"]), 3),
            _r(router["route_plan_fused_us"], 3),
            1 if gemm_uses_pair(wl.R, wl.E) else 0]
     run.free()
@@ -747,6 +793,11 @@ def run_ours(args):
     fp8_info["how"] = ("moe_ffn_fused_fp8 (h and W2 in E4M3, per-row / per-column fp32 scales), "
                        "L2 flushed before each step; the GEMM2 rate on the quantised h of a "
                        "stage-by-stage pass")
+    mx_info = run.mx_leg(args.steps, args.warmup)
+    mx_info["how"] = ("moe_ffn_fused_mx (h quantised in GEMM1's SwiGLU epilogue, one power-of-two "
+                      "scale per 32 values along K; W2 likewise, offline; tcgen05 "
+                      "kind::mxf8f6f4.block_scale), L2 flushed before each step; GEMM times from "
+                      "the library's stage events in separate steps")
     e2e_ms, h2d, d2h = run.e2e_ms(args.steps, barrier)
     run.free()
 
@@ -788,6 +839,9 @@ def run_ours(args):
     fp8_info["gemm2_e4m3_frac_of_fp8_peak"] = fp8_info["gemm2_e4m3_tflops"] / (2.0 * peak)
     fp8_info["fp8_peak_tflops"] = 2.0 * peak
     fp8_info["tokens_per_s"] = D.whole_job_rate(M, 1, fp8_info["ms_per_step"] / 1e3)
+    mx_info["gemm2_mx_frac_of_fp8_peak"] = mx_info["gemm2_mx_tflops"] / (2.0 * peak)
+    mx_info["gemm1_frac"] = mx_info["gemm1_mx_tflops"] / peak
+    mx_info["tokens_per_s"] = D.whole_job_rate(M, 1, mx_info["ms_per_step"] / 1e3)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -836,6 +890,7 @@ def run_ours(args):
             "layer_tflops": wl.flops() / (ms_per_step / 1e3) / 1e12,
             "router_plan_us": router_us,
             "fp8_layer": fp8_info,
+            "mx_layer": mx_info,
             # last, so that they stay in view at the end of the line: one record per
             # other workload, columns as named (fractions of the measured burst
             # peaks; fp8 fraction of 2x the bf16 peak; pair = CTA-pair GEMM kernel)

@@ -25,8 +25,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
 
 EPI_STORE, EPI_SWIGLU, EPI_WEIGHT_SCATTER = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024   # MOE_NOALLOC_SCRATCH_BYTES
-OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FFN_FP8 = \
-    0, 1, 2, 3, 4, 5, 6
+(OP_PLAN, OP_DISPATCH, OP_GROUPED_GEMM, OP_COMBINE, OP_FFN_FUSED, OP_ROUTE, OP_FFN_FP8,
+ OP_GEMM_MX, OP_FFN_MX) = range(9)
 
 # Every symbol include/moe.h declares.
 EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_route_plan", "moe_plan",
@@ -35,7 +35,9 @@ EXPORTS = ["moe_abi_version", "moe_workspace_size", "moe_route", "moe_route_plan
            "moe_ffn_fused_add", "moe_ffn_fused_noalloc",
            "moe_get_device_status", "moe_set_wait_timeout_ns", "moe_set_fault_injection",
            "moe_set_stage_events", "moe_quantize_weights_e4m3", "moe_quantize_rows_e4m3",
-           "moe_grouped_gemm_e4m3", "moe_ffn_fused_fp8", "moe_last_error"]
+           "moe_grouped_gemm_e4m3", "moe_ffn_fused_fp8", "moe_quantize_weights_mx",
+           "moe_quantize_rows_mx", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_mx",
+           "moe_ffn_fused_mx", "moe_last_error"]
 
 
 class MoEError(RuntimeError):
@@ -103,6 +105,17 @@ def load(path: str | None = None):
     lib.moe_ffn_fused_fp8.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P, sz,
                                       P]
     lib.moe_ffn_fused_fp8.restype = st
+    lib.moe_quantize_weights_mx.argtypes = [P, i32, i64, i64, P, P, P]
+    lib.moe_quantize_weights_mx.restype = st
+    lib.moe_quantize_rows_mx.argtypes = [P, i64, i64, P, P, P]
+    lib.moe_quantize_rows_mx.restype = st
+    lib.moe_grouped_gemm_swiglu_mx.argtypes = [P, P, P, i32, i64, i64, i64, P, P, P, sz, P]
+    lib.moe_grouped_gemm_swiglu_mx.restype = st
+    lib.moe_grouped_gemm_mx.argtypes = [P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, sz, P]
+    lib.moe_grouped_gemm_mx.restype = st
+    lib.moe_ffn_fused_mx.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P, sz,
+                                     P]
+    lib.moe_ffn_fused_mx.restype = st
     lib.moe_set_stage_events.argtypes = [P]
     lib.moe_set_stage_events.restype = st
     lib.moe_last_error.restype = ctypes.c_char_p
@@ -275,6 +288,56 @@ def moe_ffn_fused_fp8(x, W1, W2q, w2_scale, topk_ids, topk_w, out, counts, offse
                                     _ptr(topk_w), M, H, F2 // 2, E, topk, _ptr(out), _ptr(counts),
                                     _ptr(offsets), _ptr(perm), _ptr(ws), ws.numel(),
                                     _stream(stream)))
+
+
+def moe_quantize_weights_mx(W, BqT, sf, stream=None):
+    """W bf16 [E, K, N] -> BqT uint8 [E, N, K] (E4M3 codes, K contiguous), sf uint8
+    [E, N, K / 32] (block scale codes e + 127)."""
+    E, K, N = W.shape
+    _check(load().moe_quantize_weights_mx(_ptr(W), E, K, N, _ptr(BqT), _ptr(sf), _stream(stream)))
+
+
+def moe_quantize_rows_mx(A, Aq, sf, stream=None):
+    """A bf16 [R, K] -> Aq uint8 [R, K] (E4M3 codes), sf uint8 [R, K / 32]."""
+    R, K = A.shape
+    _check(load().moe_quantize_rows_mx(_ptr(A), R, K, _ptr(Aq), _ptr(sf), _stream(stream)))
+
+
+def moe_grouped_gemm_swiglu_mx(A, B, offsets, hq, h_sf, ws, stream=None):
+    """GEMM1 + SwiGLU with h quantised in the epilogue: hq uint8 [R, N2 / 2], h_sf
+    uint8 [R, N2 / 64]."""
+    R, K = A.shape
+    E, K2, N2 = B.shape
+    if K2 != K:
+        raise ValueError(f"A has K={K} but B has K={K2}")
+    _check(load().moe_grouped_gemm_swiglu_mx(_ptr(A), _ptr(B), _ptr(offsets), E, R, K, N2,
+                                             _ptr(hq), _ptr(h_sf), _ptr(ws), ws.numel(),
+                                             _stream(stream)))
+
+
+def moe_grouped_gemm_mx(Aq, a_sf, BqT, b_sf, offsets, C, ws, w_sorted=None, perm=None,
+                        stream=None):
+    """C fp32 [R, N] from block-scaled E4M3 Aq [R, K] and BqT [E, N, K] (see include/moe.h)."""
+    R, K = Aq.shape
+    E, N, K2 = BqT.shape
+    if K2 != K:
+        raise ValueError(f"Aq has K={K} but BqT has K={K2}")
+    _check(load().moe_grouped_gemm_mx(_ptr(Aq), _ptr(a_sf), _ptr(BqT), _ptr(b_sf), _ptr(offsets),
+                                      E, R, K, N, _ptr(w_sorted), _ptr(perm), _ptr(C), _ptr(ws),
+                                      ws.numel(), _stream(stream)))
+
+
+def moe_ffn_fused_mx(x, W1, W2q, w2_sf, topk_ids, topk_w, out, counts, offsets, perm, ws,
+                     stream=None):
+    """The layer with the block-scaled E4M3 down projection; W2q / w2_sf from
+    moe_quantize_weights_mx."""
+    M, H = x.shape
+    E, _, F2 = W1.shape
+    topk = topk_ids.shape[1]
+    _check(load().moe_ffn_fused_mx(_ptr(x), _ptr(W1), _ptr(W2q), _ptr(w2_sf), _ptr(topk_ids),
+                                   _ptr(topk_w), M, H, F2 // 2, E, topk, _ptr(out), _ptr(counts),
+                                   _ptr(offsets), _ptr(perm), _ptr(ws), ws.numel(),
+                                   _stream(stream)))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

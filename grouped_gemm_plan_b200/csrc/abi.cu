@@ -48,6 +48,27 @@ int launch_moe_layer(const void* x, const void* W1, const void* W2, const int32_
                      int32_t n_c, int32_t* status, void* sync_area, uint64_t timeout_ns,
                      int32_t withhold_mtile, int num_sms, cudaStream_t stream);
 int32_t profiled_n_c(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk);
+int launch_grouped_gemm_swiglu_mx(const void* A, const void* B, const int32_t* offsets, int32_t E,
+                                  int64_t R, int64_t K, int64_t N2, uint8_t* q, uint8_t* sf,
+                                  bool sf_row_major, int32_t kg_pad, int32_t* status,
+                                  uint64_t timeout_ns, int num_sms, cudaStream_t stream);
+int32_t mx_kg_pad(int64_t K);
+size_t mx_sfa_bytes(int64_t R, int32_t E, int64_t K);
+size_t mx_sfb_bytes(int32_t E, int64_t N, int64_t K);
+cudaError_t launch_quantize_weights_mx(const void* W, int32_t E, int64_t K, int64_t N, void* BqT,
+                                       uint8_t* sf, int num_sms, cudaStream_t stream);
+cudaError_t launch_quantize_rows_mx(const void* A, int64_t R, int64_t K, void* Aq, uint8_t* sf,
+                                    int num_sms, cudaStream_t stream);
+cudaError_t launch_pack_sfa(const uint8_t* sf, const int32_t* offsets, int32_t E, int64_t R,
+                            int64_t K, uint8_t* groups, int32_t* status, int num_sms,
+                            cudaStream_t stream);
+cudaError_t launch_pack_sfb(const uint8_t* sf, int32_t E, int64_t N, int64_t K, uint8_t* groups,
+                            int num_sms, cudaStream_t stream);
+int launch_grouped_gemm_mx(const void* Aq, const uint8_t* sfa_groups, const void* BqT,
+                           const uint8_t* sfb_groups, const int32_t* offsets, int32_t E, int64_t R,
+                           int64_t K, int64_t N, const float* w_sorted, const int32_t* perm,
+                           float* C, int32_t* status, uint64_t timeout_ns, int num_sms,
+                           cudaStream_t stream);
 cudaError_t launch_route(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* ids,
                          float* w, int num_sms, cudaStream_t stream);
 cudaError_t launch_route_plan(const float* logits, int64_t M, int32_t E, int32_t topk, int32_t* ids,
@@ -158,6 +179,51 @@ Fp8Layout fp8_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
   return L;
 }
 
+// moe_grouped_gemm_mx: the control block, then the A and B scale groups.
+struct GemmMxLayout {
+  size_t sfa, sfb, total;
+};
+
+GemmMxLayout gemm_mx_layout(int64_t R, int64_t N, int64_t K, int32_t E) {
+  GemmMxLayout L;
+  size_t off = kCtrlBytes;
+  L.sfa = off;
+  off += align256(moe::mx_sfa_bytes(R, E, K));
+  L.sfb = off;
+  off += align256(moe::mx_sfb_bytes(E, N, K));
+  L.total = off;
+  return L;
+}
+
+// moe_ffn_fused_mx: plan scratch, the dispatched rows, the E4M3 codes of h and
+// their scale groups (written by GEMM1's epilogue), the weights' scale groups, the
+// weighted rows (fp32), sorted gate weights and the token-order slots.
+struct MxLayout {
+  size_t xp, hq, sfa, sfb, yk, w_sorted, inv, total;
+};
+
+MxLayout mx_layout(int64_t M, int64_t H, int64_t F, int32_t E, int32_t topk) {
+  const int64_t R = M * topk;
+  MxLayout L;
+  size_t off = kCtrlBytes + plan_scratch_bytes(E);
+  L.xp = off;
+  off += align256(size_t(R) * size_t(H) * 2);
+  L.hq = off;
+  off += align256(size_t(R) * size_t(F));
+  L.sfa = off;
+  off += align256(moe::mx_sfa_bytes(R, E, F));
+  L.sfb = off;
+  off += align256(moe::mx_sfb_bytes(E, H, F));
+  L.yk = off;
+  off += align256(size_t(R) * size_t(H) * 4);
+  L.w_sorted = off;
+  off += align256(size_t(R) * 4);
+  L.inv = off;
+  off += align256(size_t(R) * 4);
+  L.total = off;
+  return L;
+}
+
 moe_status check_ws(moe_op op, void* ws, size_t ws_bytes, int64_t M, int64_t H, int64_t F,
                     int32_t E, int32_t topk) {
   if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
@@ -243,6 +309,8 @@ size_t moe_workspace_size(moe_op op, int64_t M, int64_t H, int64_t F, int32_t E,
     return SIZE_MAX;
   if (op == MOE_OP_FFN_FUSED) return fused_layout(M, H, F, E, topk).total;
   if (op == MOE_OP_FFN_FP8) return fp8_layout(M, H, F, E, topk).total;
+  if (op == MOE_OP_FFN_MX) return mx_layout(M, H, F, E, topk).total;
+  if (op == MOE_OP_GEMM_MX) return gemm_mx_layout(M, H, F, E).total;
   if (op == MOE_OP_PLAN) return kCtrlBytes + plan_scratch_bytes(E);
   return kCtrlBytes;
 }
@@ -636,6 +704,159 @@ moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
                               : cuda_fail(cudaGetLastError(), "moe_ffn_fused_fp8 GEMM2");
   err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_fp8 combine");
+  return MOE_OK;
+}
+
+moe_status moe_quantize_weights_mx(const void* W, int32_t E, int64_t K, int64_t N, void* BqT,
+                                   uint8_t* sf, void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (K <= 0 || K % 32 != 0 || N <= 0 || N % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 32 and N = %lld of 16", (long long)K, (long long)N);
+  if (K > kMaxRows || N > kMaxRows || int64_t(E) * N > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N too large");
+  if (W == nullptr || BqT == nullptr || sf == nullptr) return fail(MOE_ERR_INVALID_ARG, "W, BqT and sf must not be NULL");
+  if (!aligned16(W) || !aligned16(BqT)) return fail(MOE_ERR_MISALIGNED, "W and BqT must be 16-byte aligned");
+  const cudaError_t err = moe::launch_quantize_weights_mx(W, E, K, N, BqT, sf, num_sms_current(),
+                                                          reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_weights_mx");
+}
+
+moe_status moe_quantize_rows_mx(const void* A, int64_t R, int64_t K, void* Aq, uint8_t* sf,
+                                void* stream) {
+  g_last_error.clear();
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 32 != 0 || K > (int64_t(1) << 30))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 32", (long long)K);
+  if (R == 0) return MOE_OK;
+  if (A == nullptr || Aq == nullptr || sf == nullptr) return fail(MOE_ERR_INVALID_ARG, "A, Aq and sf must not be NULL");
+  if (!aligned16(A) || !aligned16(Aq)) return fail(MOE_ERR_MISALIGNED, "A and Aq must be 16-byte aligned");
+  const cudaError_t err = moe::launch_quantize_rows_mx(A, R, K, Aq, sf, num_sms_current(),
+                                                       reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_rows_mx");
+}
+
+moe_status moe_grouped_gemm_swiglu_mx(const void* A, const void* B, const int32_t* offsets,
+                                      int32_t E, int64_t R, int64_t K, int64_t N2, void* hq,
+                                      uint8_t* h_sf, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64", (long long)K);
+  if (N2 <= 0 || N2 % 128 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "N2 = %lld must be a positive multiple of 128", (long long)N2);
+  if (K > (int64_t(1) << 30) || N2 > (int64_t(1) << 30) || E * K > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N2 too large");
+  moe_status st = check_ws(MOE_OP_GROUPED_GEMM, ws, ws_bytes, R, N2, K, E, 1);
+  if (st != MOE_OK) return st;
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets must not be NULL");
+  if (R == 0) return MOE_OK;
+  if (A == nullptr || B == nullptr || hq == nullptr || h_sf == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "A, B, hq and h_sf must not be NULL");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(hq)) return fail(MOE_ERR_MISALIGNED, "A, B and hq must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(h_sf) & 1u) != 0) return fail(MOE_ERR_MISALIGNED, "h_sf must be 2-byte aligned");
+  const int rc = moe::launch_grouped_gemm_swiglu_mx(A, B, offsets, E, R, K, N2, static_cast<uint8_t*>(hq),
+                                                    h_sf, true, 0, status_word(ws), g_timeout_ns,
+                                                    num_sms_current(), reinterpret_cast<cudaStream_t>(stream));
+  if (rc == 1) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_grouped_gemm_swiglu_mx launch");
+  return MOE_OK;
+}
+
+moe_status moe_grouped_gemm_mx(const void* Aq, const uint8_t* a_sf, const void* BqT,
+                               const uint8_t* b_sf, const int32_t* offsets, int32_t E, int64_t R,
+                               int64_t K, int64_t N, const float* w_sorted, const int32_t* perm,
+                               float* C, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  if (E < 1 || E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E = %d not in [1, %d]", E, MOE_MAX_EXPERTS);
+  if (R < 0 || R > kMaxRows) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (K <= 0 || K % 32 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 32", (long long)K);
+  if (N <= 0 || N % 64 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "N = %lld must be a positive multiple of 64", (long long)N);
+  if (K > (int64_t(1) << 30) || N > (int64_t(1) << 30) || int64_t(E) * N > kMaxRows)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "K or N too large");
+  moe_status st = check_ws(MOE_OP_GEMM_MX, ws, ws_bytes, R, N, K, E, 1);
+  if (st != MOE_OK) return st;
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets must not be NULL");
+  if (R == 0) return MOE_OK;
+  if (Aq == nullptr || BqT == nullptr || C == nullptr || a_sf == nullptr || b_sf == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "Aq, a_sf, BqT, b_sf and C must not be NULL");
+  if (!aligned16(Aq) || !aligned16(BqT) || !aligned16(C))
+    return fail(MOE_ERR_MISALIGNED, "Aq, BqT and C must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const GemmMxLayout L = gemm_mx_layout(R, N, K, E);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int sms = num_sms_current();
+  cudaError_t err = moe::launch_pack_sfa(a_sf, offsets, E, R, K, base + L.sfa, status_word(ws), sms, s);
+  if (err == cudaSuccess) err = moe::launch_pack_sfb(b_sf, E, N, K, base + L.sfb, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_grouped_gemm_mx scale packing");
+  const int rc = moe::launch_grouped_gemm_mx(Aq, base + L.sfa, BqT, base + L.sfb, offsets, E, R, K, N,
+                                             w_sorted, perm, C, status_word(ws), g_timeout_ns, sms, s);
+  if (rc == 1) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  if (rc != 0) return cuda_fail(cudaGetLastError(), "moe_grouped_gemm_mx launch");
+  return MOE_OK;
+}
+
+moe_status moe_ffn_fused_mx(const void* x, const void* W1, const void* W2q, const uint8_t* w2_sf,
+                            const int32_t* topk_ids, const float* topk_w, int64_t M, int64_t H,
+                            int64_t F, int32_t E, int32_t topk, void* out, int32_t* counts,
+                            int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                            void* stream) {
+  g_last_error.clear();
+  moe_status st = moe::check_layer_shape(M, H, F, E, topk);
+  if (st != MOE_OK) return st;
+  st = check_ws(MOE_OP_FFN_MX, ws, ws_bytes, M, H, F, E, topk);
+  if (st != MOE_OK) return st;
+  if (counts == nullptr || offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current();
+  if (M == 0) {
+    cudaError_t err = moe::launch_plan(topk_ids, topk_w, 0, E, counts, offsets, perm, nullptr,
+                                       nullptr, status_word(ws), plan_scratch(ws), sms, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ffn_fused_mx plan");
+  }
+  if (x == nullptr || W1 == nullptr || W2q == nullptr || w2_sf == nullptr || topk_ids == nullptr ||
+      topk_w == nullptr || out == nullptr || perm == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "x, W1, W2q, w2_sf, topk_ids, topk_w, out and perm must not be NULL");
+  if (!aligned16(x) || !aligned16(W1) || !aligned16(W2q) || !aligned16(out))
+    return fail(MOE_ERR_MISALIGNED, "x, W1, W2q and out must be 16-byte aligned");
+  const int64_t R = M * topk;
+  moe::PdlScope pdl(static_cast<double>(R) * static_cast<double>(H) * static_cast<double>(F) <
+                    4294967296.0);
+  const MxLayout L = mx_layout(M, H, F, E, topk);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* xp = base + L.xp;
+  uint8_t* hq = base + L.hq;
+  uint8_t* sfa = base + L.sfa;
+  uint8_t* sfb = base + L.sfb;
+  float* yk = reinterpret_cast<float*>(base + L.yk);
+  float* w_sorted = reinterpret_cast<float*>(base + L.w_sorted);
+  int32_t* inv = reinterpret_cast<int32_t*>(base + L.inv);
+  int32_t* status = status_word(ws);
+
+  // stage events (moe_set_stage_events): the first stage holds the weight-scale
+  // rearrangement and the plan
+  stage_mark(0, s);
+  cudaError_t err = moe::launch_pack_sfb(w2_sf, E, H, F, sfb, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_mx weight scales");
+  err = moe::launch_plan(topk_ids, topk_w, static_cast<int32_t>(R), E, counts, offsets, perm, inv,
+                         w_sorted, status, plan_scratch(ws), sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_mx plan");
+  stage_mark(1, s);
+  err = moe::launch_dispatch_tokens(x, inv, M, H, topk, xp, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_mx dispatch");
+  stage_mark(2, s);
+  int rc = moe::launch_grouped_gemm_swiglu_mx(xp, W1, offsets, E, R, H, 2 * F, hq, sfa, false,
+                                              moe::mx_kg_pad(F), status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (GEMM1)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused_mx GEMM1");
+  stage_mark(3, s);
+  rc = moe::launch_grouped_gemm_mx(hq, sfa, W2q, sfb, offsets, E, R, F, H, w_sorted, perm, yk,
+                                   status, g_timeout_ns, sms, s);
+  if (rc != 0) return rc == 1 ? fail(MOE_ERR_CUDA, "tensor map encode failed (MX GEMM2)")
+                              : cuda_fail(cudaGetLastError(), "moe_ffn_fused_mx GEMM2");
+  stage_mark(4, s);
+  err = moe::launch_combine(yk, true, nullptr, nullptr, M, H, topk, out, status, sms, s);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ffn_fused_mx combine");
+  stage_mark(5, s);
   return MOE_OK;
 }
 

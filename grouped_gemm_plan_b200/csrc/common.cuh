@@ -21,6 +21,11 @@
 
 namespace moe {
 
+// Epilogue of the SwiGLU GEMM that writes block-scaled E4M3 codes of h and their
+// scale exponents (internal: reached through moe_grouped_gemm_swiglu_mx and the
+// MX layer, not through moe_grouped_gemm's epilogue argument).
+constexpr int EPI_SWIGLU_MX = 3;
+
 // ---------------------------------------------------------------- status word
 
 // First error wins: a kernel never overwrites an earlier device error.

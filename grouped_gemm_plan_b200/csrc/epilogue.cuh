@@ -13,6 +13,8 @@
 // are free of bank conflicts.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -39,6 +41,25 @@ __device__ __forceinline__ void warp_store_rows128(const uint4 (&seg)[8], uint8_
   }
 }
 
+// The same for 64-byte row segments (slot j of row r at r * 4 + (j ^ ((r >> 1) & 3)):
+// conflict-free both ways); four lanes cover one row's 64 bytes, eight rows per
+// store instruction.
+__device__ __forceinline__ void warp_store_rows64(const uint4* seg, uint8_t* dst, uint4* buf, int lane) {
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) buf[lane * 4 + (j ^ ((lane >> 1) & 3))] = seg[j];
+  __syncwarp();
+  const unsigned long long mine = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int row = it * 8 + (lane >> 2);
+    const int c16 = lane & 3;
+    const unsigned long long d = __shfl_sync(0xffffffffu, mine, row);
+    const uint4 v = buf[row * 4 + (c16 ^ ((row >> 1) & 3))];
+    if (d != 0ull) reinterpret_cast<uint4*>(d)[c16] = v;
+  }
+}
+
 __device__ __forceinline__ void pack8_bf16(const float* v, float scale, uint4& out) {
   out.x = pack_bf16x2(v[0] * scale, v[1] * scale);
   out.y = pack_bf16x2(v[2] * scale, v[3] * scale);
@@ -54,6 +75,84 @@ __device__ __forceinline__ void pack8_swiglu(const float* g, const float* u, uin
   out.y = pack_bf16x2(silu_fast(g[2]) * u[2], silu_fast(g[3]) * u[3]);
   out.z = pack_bf16x2(silu_fast(g[4]) * u[4], silu_fast(g[5]) * u[5]);
   out.w = pack_bf16x2(silu_fast(g[6]) * u[6], silu_fast(g[7]) * u[7]);
+}
+
+// ---------------------------------------------------------------- block-scaled E4M3 (MX)
+// Blocks of 32 consecutive h values of a row share one power-of-two scale 2^e, e
+// the smallest integer with amax <= 448 * 2^e (448: the largest E4M3 value),
+// stored as the E8M0 code e + 127; the elements are q = E4M3(v * 2^-e), nearest,
+// ties to even.  (The PTO MegaMoE article, section "MegaMoE 融合算子七阶段": SwiGLU
+// quantises each segment it consumes; the block size and scale format are those of
+// the tcgen05 block-scaled MMA.)
+
+// e of a block with largest magnitude `amax` >= 0, clamped to [-127, 127] (-127
+// for an all-zero block), from the bits of amax = m * 2^p, m in [1, 2): since
+// 448 = 1.75 * 2^8, e = p - 8 when m <= 1.75, else p - 7.  Below 2^-126 (zero or
+// subnormal) e would be at most -134, which clamps to -127.
+__device__ __forceinline__ int mx_exponent_of(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int biased = static_cast<int>(b >> 23);
+  if (biased == 0) return -127;
+  const int e = biased - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3)) |
+         (static_cast<uint32_t>(__nv_cvt_float_to_fp8(b, __NV_SATFINITE, __NV_E4M3)) << 8) |
+         (static_cast<uint32_t>(__nv_cvt_float_to_fp8(c, __NV_SATFINITE, __NV_E4M3)) << 16) |
+         (static_cast<uint32_t>(__nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3)) << 24);
+}
+
+// 32 values -> their 32 codes (value i in byte i of lo:hi) and the block's scale
+// code e + 127 (returned).  v * 2^-e is exact in fp32 (a power-of-two scaling
+// that stays at or below 448), so the only rounding is the E4M3 one.
+__device__ __forceinline__ uint32_t mx_block32(const float* v, uint4& lo, uint4& hi) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  const int e = mx_exponent_of(m);
+  const int es = e > 126 ? 126 : e;
+  const float s = __uint_as_float(static_cast<uint32_t>(127 - es) << 23);  // 2^-e
+  uint32_t w[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    w[k] = e4m3x4(v[4 * k] * s, v[4 * k + 1] * s, v[4 * k + 2] * s, v[4 * k + 3] * s);
+  lo = make_uint4(w[0], w[1], w[2], w[3]);
+  hi = make_uint4(w[4], w[5], w[6], w[7]);
+  return static_cast<uint32_t>(e + 127);
+}
+
+// SwiGLU + block-scaled E4M3 of `nseg` (1 or 2) segments of 64 h columns of this
+// warp's 32 rows: segment c takes gate columns [64c, 64c + 64) and up columns
+// up_off + [64c, 64c + 64) of the accumulator and holds two blocks of 32 h values.
+// The 64 * nseg code bytes of a row go to row_dst (nullptr: not written).
+// Returns the scale codes of the 2 * nseg blocks, block b in byte b.
+// Warp-collective.
+__device__ __forceinline__ uint32_t epilogue_swiglu_mx(uint32_t t_row, uint8_t* row_dst, int nseg,
+                                                       uint32_t up_off, uint4* buf, int lane) {
+  uint4 seg[8];
+  uint32_t codes = 0;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (c >= nseg) break;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float g[32], u[32];
+      tmem_ld32(t_row + c * 64 + half * 32, g);
+      tmem_ld32(t_row + up_off + c * 64 + half * 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = silu_fast(g[i]) * u[i];
+      const uint32_t code = mx_block32(g, seg[4 * c + 2 * half], seg[4 * c + 2 * half + 1]);
+      codes |= code << (8 * (2 * c + half));
+    }
+  }
+  if (nseg == 2)
+    warp_store_rows128(seg, row_dst, buf, lane);
+  else
+    warp_store_rows64(seg, row_dst, buf, lane);
+  return codes;
 }
 
 // The epilogue of `nseg` 128-byte output segments of this warp's 32 rows:

@@ -82,6 +82,12 @@ struct Gemm2Args {
   __nv_bfloat16* C;
   float* Cf;
   int64_t ldc;
+  // EPI_SWIGLU_MX: E4M3 codes of h [R, ldc] and their scale codes, row-major
+  // [R, sf_ld] (sf_ld > 0) or in the 512-byte groups the block-scaled down
+  // projection loads (sf_ld = 0; kg_pad groups of 128 columns per 128-row block)
+  uint8_t* q;
+  uint8_t* sf;
+  int32_t sf_ld, kg_pad;
   int32_t* status;
   int32_t* queue;      // [0] ticket counter, [1] CTAs finished (both zero between launches)
   uint64_t timeout_ns;
@@ -169,6 +175,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_tstart[MOE_MAX_EXPERTS + 1];
 
+  constexpr bool kSwiglu = EPI == MOE_EPI_SWIGLU || EPI == EPI_SWIGLU_MX;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t E = args.E;
   const uint32_t rank = cluster_rank();
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           tma2_load_2d(sa + c * P_A_BOX_BYTES, tc.m128 ? &tmA64 : &tmA, fb, kb * P_BK + 64 * c, arow);
         for (int b = 0; b < nbox; ++b) {
           int32_t n;
-          if (EPI == MOE_EPI_SWIGLU) {
+          if (kSwiglu) {
             const int32_t j0 = tc.ni * 128;
             if (half)            // leader: gate, peer: up, 64 columns of the half
               n = (rank == 0 ? 0 : args.up_col) + j0 + 64 * h;
@@ -470,7 +477,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       if (tc.m128) {
         r = 64 * static_cast<int32_t>(rank) + 32 * (q & 1) + lane;
         const int32_t nh = q >> 1;       // lanes [64, 128) hold accumulator columns [128, 256)
-        if (EPI == MOE_EPI_SWIGLU) {
+        if (kSwiglu) {
           col0 = tc.ni * 128 + 64 * nh;
           nseg = 1;
           up_off = 64;
@@ -481,7 +488,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         }
       } else {
         r = 128 * static_cast<int32_t>(rank) + 32 * q + lane;
-        if (EPI == MOE_EPI_SWIGLU) {
+        if (kSwiglu) {
           col0 = tc.ni * 128 + (var != V_WHOLE ? 64 * h : 0);
           nseg = var != V_WHOLE ? 1 : 2;
           up_off = var != V_WHOLE ? 64 : 128;
@@ -506,6 +513,33 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         }
         epilogue_segments<MOE_EPI_WEIGHT_SCATTER>(t_row, dst, args.n_out - col0, nseg, 0, scale,
                                                   stage_buf, lane);
+      } else if (EPI == EPI_SWIGLU_MX) {
+        // h columns past F (F an odd multiple of 64: the last column tile is half
+        // used) are neither computed nor written
+        const int32_t n_left = args.n_out - col0;
+        const int ns = n_left >= 64 * nseg ? nseg : (n_left > 0 ? 1 : 0);
+        uint8_t* dst = row_ok ? args.q + static_cast<int64_t>(s) * args.ldc + col0 : nullptr;
+        const uint32_t codes = ns > 0 ? epilogue_swiglu_mx(t_row, dst, ns, up_off, stage_buf, lane) : 0u;
+        if (row_ok) {
+          // two scale codes (one 64-column segment) per 16-bit store
+          const int32_t kb0 = col0 / 32;
+          for (int c = 0; c < ns; ++c) {
+            const int32_t kb = kb0 + 2 * c;
+            const uint16_t v = static_cast<uint16_t>(codes >> (16 * c));
+            uint8_t* p;
+            if (args.sf_ld > 0) {
+              p = args.sf + static_cast<int64_t>(s) * args.sf_ld + kb;
+            } else {
+              // group (m-tile gm, 128-row half, 128 columns kb / 4): row i + 32 j of the
+              // half and its block b of the group at byte 16 i + 4 j + b
+              const int32_t gm = s_tstart[tc.e] / args.n_tiles_n + (tc.row0 - s_off[tc.e]) / P_BM;
+              const int32_t ri = r & 127;
+              p = args.sf + (static_cast<int64_t>(gm * 2 + (r >> 7)) * args.kg_pad + kb / 4) * 512 +
+                  16 * (ri & 31) + 4 * (ri >> 5) + (kb & 3);
+            }
+            *reinterpret_cast<uint16_t*>(p) = v;
+          }
+        }
       } else {
         uint8_t* dst = row_ok ? reinterpret_cast<uint8_t*>(args.C + static_cast<int64_t>(s) * args.ldc + col0)
                               : nullptr;
@@ -564,6 +598,50 @@ static cudaError_t launch2_t(int grid, const CUtensorMap& a, const CUtensorMap& 
                     P_DYN_SMEM, stream, 2, a, a64, b, args);
 }
 
+// Tensor maps, arguments and grid of one launch; false if a tensor map cannot be
+// encoded.  `swiglu`: B holds gate | up column halves of N / 2 each.
+static bool prepare2(const void* A, const void* B, const int32_t* offsets, int32_t E, int64_t R,
+                     int64_t K, int64_t N, bool swiglu, int32_t* status, uint64_t timeout_ns,
+                     int num_sms, CUtensorMap* tmA, CUtensorMap* tmA64, CUtensorMap* tmB,
+                     Gemm2Args* a, int* grid) {
+  const cuuint64_t adims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(R)};
+  const cuuint64_t astr[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t abox[2] = {64, 128};
+  const cuuint32_t abox64[2] = {64, 64};
+  const cuuint64_t bdims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
+                               static_cast<cuuint64_t>(E)};
+  const cuuint64_t bstr[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(K * N) * 2};
+  const cuuint32_t bbox[3] = {64, P_BK, 1};
+  if (!enc2(tmA, 2, A, adims, astr, abox) || !enc2(tmA64, 2, A, adims, astr, abox64) ||
+      !enc2(tmB, 3, B, bdims, bstr, bbox))
+    return false;
+  *a = Gemm2Args{};
+  a->offsets = offsets;
+  a->E = E;
+  a->R = static_cast<int32_t>(R);
+  a->K = static_cast<int32_t>(K);
+  a->status = status;
+  a->queue = status + 32;
+  a->timeout_ns = timeout_ns;
+  if (swiglu) {
+    a->n_out = static_cast<int32_t>(N / 2);
+    a->up_col = static_cast<int32_t>(N / 2);
+    a->n_tiles_n = static_cast<int32_t>((N / 2 + 127) / 128);
+    a->ldc = N / 2;
+  } else {
+    a->n_out = static_cast<int32_t>(N);
+    a->up_col = 0;
+    a->n_tiles_n = static_cast<int32_t>((N + P_BN - 1) / P_BN);
+    a->ldc = N;
+  }
+  const int64_t tiles_max = (R / P_BM + (E < R ? E : R)) * a->n_tiles_n;
+  int64_t pairs = num_sms / 2;
+  if (2 * tiles_max < pairs) pairs = 2 * tiles_max;   // the last tiles run as two halves
+  if (pairs < 1) pairs = 1;
+  *grid = static_cast<int>(2 * pairs);
+  return true;
+}
+
 // Same contract as launch_grouped_gemm (0 ok, 1 tensor map, 2 CUDA error).  `status`
 // is the workspace's status word; the tile queue lives at status + 32 (byte 128 of
 // the workspace's 256-byte control block).
@@ -573,45 +651,15 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
                             int num_sms, cudaStream_t stream) {
   if (R == 0) return 0;
   CUtensorMap tmA, tmA64, tmB;
-  const cuuint64_t adims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(R)};
-  const cuuint64_t astr[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t abox[2] = {64, 128};
-  const cuuint32_t abox64[2] = {64, 64};
-  const cuuint64_t bdims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K),
-                               static_cast<cuuint64_t>(E)};
-  const cuuint64_t bstr[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(K * N) * 2};
-  const cuuint32_t bbox[3] = {64, P_BK, 1};
-  if (!enc2(&tmA, 2, A, adims, astr, abox) || !enc2(&tmA64, 2, A, adims, astr, abox64) ||
-      !enc2(&tmB, 3, B, bdims, bstr, bbox))
-    return 1;
   Gemm2Args a;
-  a.offsets = offsets;
-  a.E = E;
-  a.R = static_cast<int32_t>(R);
-  a.K = static_cast<int32_t>(K);
+  int grid = 0;
+  if (!prepare2(A, B, offsets, E, R, K, N, epi == MOE_EPI_SWIGLU, status, timeout_ns, num_sms, &tmA,
+                &tmA64, &tmB, &a, &grid))
+    return 1;
   a.w_sorted = w_sorted;
   a.perm = perm;
   a.C = static_cast<__nv_bfloat16*>(C);
   a.Cf = static_cast<float*>(C);
-  a.status = status;
-  a.queue = status + 32;
-  a.timeout_ns = timeout_ns;
-  if (epi == MOE_EPI_SWIGLU) {
-    a.n_out = static_cast<int32_t>(N / 2);
-    a.up_col = static_cast<int32_t>(N / 2);
-    a.n_tiles_n = static_cast<int32_t>((N / 2 + 127) / 128);
-    a.ldc = N / 2;
-  } else {
-    a.n_out = static_cast<int32_t>(N);
-    a.up_col = 0;
-    a.n_tiles_n = static_cast<int32_t>((N + P_BN - 1) / P_BN);
-    a.ldc = N;
-  }
-  const int64_t tiles_max = (R / P_BM + (E < R ? E : R)) * a.n_tiles_n;
-  int64_t pairs = num_sms / 2;
-  if (2 * tiles_max < pairs) pairs = 2 * tiles_max;   // the last tiles run as two halves
-  if (pairs < 1) pairs = 1;
-  const int grid = static_cast<int>(2 * pairs);
   cudaError_t err;
   if (epi == MOE_EPI_SWIGLU)
     err = launch2_t<MOE_EPI_SWIGLU>(grid, tmA, tmA64, tmB, a, stream);
@@ -620,6 +668,28 @@ int launch_grouped_gemm_2sm(const void* A, const void* B, const int32_t* offsets
   else
     err = launch2_t<MOE_EPI_STORE>(grid, tmA, tmA64, tmB, a, stream);
   return err == cudaSuccess ? 0 : 2;
+}
+
+// GEMM1 with the SwiGLU + block-scaled E4M3 epilogue: B = W1 [E, K, N2] (gate |
+// up), q [R, N2 / 2] codes, sf their scale codes, row-major [R, N2 / 64] when
+// sf_row_major, else in the 512-byte groups of the MX down projection (kg_pad
+// groups per 128-row block).  Same return contract as launch_grouped_gemm_2sm.
+int launch_grouped_gemm_swiglu_mx(const void* A, const void* B, const int32_t* offsets, int32_t E,
+                                  int64_t R, int64_t K, int64_t N2, uint8_t* q, uint8_t* sf,
+                                  bool sf_row_major, int32_t kg_pad, int32_t* status,
+                                  uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+  if (R == 0) return 0;
+  CUtensorMap tmA, tmA64, tmB;
+  Gemm2Args a;
+  int grid = 0;
+  if (!prepare2(A, B, offsets, E, R, K, N2, true, status, timeout_ns, num_sms, &tmA, &tmA64, &tmB,
+                &a, &grid))
+    return 1;
+  a.q = q;
+  a.sf = sf;
+  a.sf_ld = sf_row_major ? static_cast<int32_t>(N2 / 64) : 0;
+  a.kg_pad = kg_pad;
+  return launch2_t<EPI_SWIGLU_MX>(grid, tmA, tmA64, tmB, a, stream) == cudaSuccess ? 0 : 2;
 }
 
 }  // namespace moe

@@ -123,5 +123,40 @@ __device__ __forceinline__ void umma2_e4m3(uint32_t tmem_d, uint64_t adesc, uint
       : "memory");
 }
 
+// Block-scaled E4M3 MMA (kind::mxf8f6f4, one E8M0 scale per 32 values of K for
+// every row of A and every column of B): the scales are read from TMEM at
+// `sfa` / `sfb`, the 32-bit TMEM addresses of the scale columns with the byte of
+// this MMA's K block in bits [30, 32); the same byte index sits in the
+// instruction descriptor (bits [29, 31) for A, [4, 6) for B).
+__device__ __forceinline__ void umma2_mx(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy of one 512-byte scale-factor group from shared memory (at the same
+// address in both CTAs) into 4 TMEM columns of every lane quarter of both CTAs:
+// source byte 16 i + 4 j + b lands in column j, byte b, of lanes i, 32 + i, 64 + i
+// and 96 + i.
+__device__ __forceinline__ void utccp2_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled operand (the scale-factor groups:
+// rows of 16 bytes, 128 bytes between 8-row core matrices).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
 }  // namespace
 }  // namespace moe

@@ -88,7 +88,9 @@ typedef enum moe_op {
   MOE_OP_COMBINE = 3,
   MOE_OP_FFN_FUSED = 4,
   MOE_OP_ROUTE = 5,
-  MOE_OP_FFN_FP8 = 6   /* moe_ffn_fused_fp8 */
+  MOE_OP_FFN_FP8 = 6,  /* moe_ffn_fused_fp8 */
+  MOE_OP_GEMM_MX = 7,  /* moe_grouped_gemm_mx: M = R, H = N, F = K */
+  MOE_OP_FFN_MX = 8    /* moe_ffn_fused_mx */
 } moe_op;
 
 /* Version of this ABI (incremented on any incompatible change). */
@@ -357,6 +359,74 @@ moe_status moe_ffn_fused_fp8(const void* x, const void* W1, const void* W2q,
                              int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- block-scaled FP8 (MX)
+ * The down projection on E4M3 with one scale per block of 32 values along the
+ * contraction ([PTO] "MegaMoE 融合算子七阶段": SwiGLU quantises each GMM1 segment
+ * it consumes; a block scale needs only the block, so GEMM1's epilogue quantises
+ * h as it computes it).  A block of 32 consecutive values along K shares the
+ * scale 2^e, e the smallest integer with (largest |v| of the block) <= 448 * 2^e,
+ * clamped to [-127, 127] (-127 for an all-zero block); the scale is stored as the
+ * byte e + 127 (E8M0); the elements are q = nearest E4M3 to v * 2^-e, ties to
+ * even.  The GEMM multiplies E4M3 blocks on the tensor core
+ * (tcgen05.mma kind::mxf8f6f4.block_scale), each block product scaled by
+ * 2^(ea + eb), and accumulates in fp32.
+ */
+
+/* moe_quantize_weights_mx -- offline, once per weight tensor:
+ *   W bf16 [E, K, N] row-major (the layout of W2, N contiguous)
+ *   BqT E4M3 bytes [E, N, K] (K contiguous), sf bytes [E, N, K / 32] (the
+ *   scale code of column n, K block b at sf[(e * N + n) * K / 32 + b]).
+ * K must be a multiple of 32, N of 16.  All pointers device, caller-owned. */
+moe_status moe_quantize_weights_mx(const void* W, int32_t E, int64_t K, int64_t N, void* BqT,
+                                   uint8_t* sf, void* stream);
+
+/* moe_quantize_rows_mx -- A bf16 [R, K] -> Aq E4M3 bytes [R, K] and sf bytes
+ * [R, K / 32] (row-major).  K must be a multiple of 32.  Rows are independent;
+ * R = 0 is a no-op. */
+moe_status moe_quantize_rows_mx(const void* A, int64_t R, int64_t K, void* Aq, uint8_t* sf,
+                                void* stream);
+
+/* moe_grouped_gemm_swiglu_mx -- GEMM1 + SwiGLU as moe_grouped_gemm with
+ * MOE_EPI_SWIGLU (A bf16 [R, K], B bf16 [E, K, N2] gate | up), with h quantised
+ * in blocks of 32 columns inside the epilogue instead of stored in bf16:
+ *   hq E4M3 bytes [R, N2 / 2], h_sf bytes [R, N2 / 64] (row-major).
+ * h is computed in fp32 from the fp32 accumulator.  N2 must be a multiple of
+ * 128, K of 64.  Workspace as for MOE_OP_GROUPED_GEMM.  Error behaviour as
+ * moe_grouped_gemm. */
+moe_status moe_grouped_gemm_swiglu_mx(const void* A, const void* B, const int32_t* offsets,
+                                      int32_t E, int64_t R, int64_t K, int64_t N2, void* hq,
+                                      uint8_t* h_sf, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_grouped_gemm_mx -- grouped GEMM on block-scaled E4M3 operands with the
+ * gate-weight scatter epilogue:
+ *   for every expert e and row s in [offsets[e], offsets[e+1]):
+ *     C[d, n] = w * sum over K blocks b of 2^(a_sf[s, b] - 127) * 2^(b_sf[e, n, b] - 127)
+ *                                       * sum_{k in b} Aq[s, k] * BqT[e, n, k]
+ *   with d = perm[s], w = w_sorted[s] (perm == NULL: d = s; w_sorted == NULL:
+ *   w = 1).  Aq [R, K] and a_sf [R, K / 32] as written by moe_quantize_rows_mx
+ *   (or moe_grouped_gemm_swiglu_mx), BqT [E, N, K] and b_sf [E, N, K / 32] as
+ *   written by moe_quantize_weights_mx; C fp32 [R, N].  K must be a multiple of
+ *   32, N of 64.  Workspace: moe_workspace_size(MOE_OP_GEMM_MX, R, N, K, E, 1)
+ *   (the scales are rearranged there into the groups the tensor core reads).
+ *   A perm entry outside [0, R) skips that row and records MOE_ERR_BAD_INDEX;
+ *   offsets inconsistent with R record it too and compute nothing. */
+moe_status moe_grouped_gemm_mx(const void* Aq, const uint8_t* a_sf, const void* BqT,
+                               const uint8_t* b_sf, const int32_t* offsets, int32_t E, int64_t R,
+                               int64_t K, int64_t N, const float* w_sorted, const int32_t* perm,
+                               float* C, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_ffn_fused_mx -- the layer with a block-scaled E4M3 down projection:
+ *   plan -> dispatch -> GEMM1 + SwiGLU with h quantised in the epilogue (codes
+ *   and scales written to the workspace; no bf16 h) -> MX GEMM2 against
+ *   (W2q, w2_sf) from moe_quantize_weights_mx on W2 [E, F, H], with the
+ *   gate-weight scatter -> combine.  Arguments as moe_ffn_fused (without n_c);
+ *   the workspace is moe_workspace_size(MOE_OP_FFN_MX, ...). */
+moe_status moe_ffn_fused_mx(const void* x, const void* W1, const void* W2q, const uint8_t* w2_sf,
+                            const int32_t* topk_ids, const float* topk_w, int64_t M, int64_t H,
+                            int64_t F, int32_t E, int32_t topk, void* out, int32_t* counts,
+                            int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                            void* stream);
+
 /* Synchronises `stream`, returns the device status word of `ws` (a moe_status)
  * and clears the control block (status word MOE_OK, tile queue zero).  Returns
  * MOE_ERR_CUDA if the stream reports an error. */
@@ -376,13 +446,14 @@ void moe_set_wait_timeout_ns(uint64_t ns);
  * Process-wide; returns MOE_ERR_INVALID_ARG for an unknown kind. */
 moe_status moe_set_fault_injection(int32_t kind, int32_t index);
 
-/* Stage timing for moe_ffn_fused (measurement only; the pages have no
- * counterpart).  events: NULL (off, the default) or an array of 6 cudaEvent_t
- * handles created by the caller; the caller keeps ownership and must keep them
- * alive while set.  While set, each moe_ffn_fused call on this thread records
+/* Stage timing for moe_ffn_fused and moe_ffn_fused_mx (measurement only; the
+ * pages have no counterpart).  events: NULL (off, the default) or an array of 6
+ * cudaEvent_t handles created by the caller; the caller keeps ownership and must
+ * keep them alive while set.  While set, each such call on this thread records
  * events[0] on its stream before the plan and events[i + 1] after stage i
  * (plan, dispatch, GEMM1 + SwiGLU, GEMM2 + scatter, combine), so that the
- * elapsed time between consecutive events is one stage's device time.  In the
+ * elapsed time between consecutive events is one stage's device time (in
+ * moe_ffn_fused_mx the first stage also rearranges the weight scales).  In the
  * single-kernel layer (n_c > 0) events[2..5] are all recorded after the layer
  * kernel.  Recording an event between two kernels serialises them, so a
  * programmatic dependent launch between those kernels no longer overlaps.
