@@ -208,8 +208,14 @@ __global__ void __launch_bounds__(256)
 // A tile's MMAs may start once the tile before it (in the other accumulator) has
 // had its shared 72 columns read out: the epilogue loads those first (columns
 // [160, 256) of accumulator 0, [0, 96) of accumulator 1), signals, then stores.
-// (An N = 128 tile needs no overlap but measured 0.34 of the fp8 peak on the
-// Phi-3.5 shape, plain E4M3 MMAs included: it pulls 1.5x the bytes per MMA.)
+// Measured alternatives, all slower on B200 (the down projection of the Phi-3.5,
+// Qwen2 and Mixtral shapes): N = 128 tiles (no overlap needed, but 0.34 of the
+// fp8 peak on Phi-3.5 with plain E4M3 MMAs too: 1.5x the bytes per MMA); M = 128
+// tiles for short experts' tails as in the bf16 GEMMs (slower on Qwen2 despite
+// the smaller padding: an M = 128 tile loads the same B bytes for half the MMA
+// work); six stages of 128 K instead of three of 256 K (6-13 % slower: twice the
+// barrier round trips and scale copies per K); copying two stages' scales at once
+// (5 % slower).
 namespace {
 constexpr int X_BM = 256;
 constexpr int X_BN = 256;
@@ -278,6 +284,14 @@ __device__ __forceinline__ XTile xdecode(int32_t t, const int32_t* s_tstart, con
 
 // One 32-column fp32 segment of this thread's row, times `scale`, through the
 // warp's staging buffer to dst (nullptr: not written).  Warp-collective.
+// Arrival on the leader's accumulator barriers: relaxed, since the MMA side needs
+// only the TMEM reads to be done (tcgen05.wait::ld precedes the arrival), not this
+// warp's global stores, which a release arrival would wait for (measured: 14 %
+// of the down projection's time on the Qwen2 shape, 2 % on Phi-3.5).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void store_seg32(const float (&v)[32], float scale, uint8_t* dst,
                                             uint4* buf, int lane) {
   uint4 seg[8];
@@ -534,7 +548,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(b ? ov_leader1 : ov_leader0);
+      if (lane == 0) mbar_arrive_cluster_relaxed(b ? ov_leader1 : ov_leader0);
       const int32_t col0 = tc.ni * X_BN;
       const int32_t n_left = args.N - col0;
       float scale = 1.0f;
@@ -566,7 +580,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(b ? te_leader1 : te_leader0);
+      if (lane == 0) mbar_arrive_cluster_relaxed(b ? te_leader1 : te_leader0);
     }
   }
 
