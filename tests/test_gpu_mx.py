@@ -284,3 +284,39 @@ def test_mx_layer_empty_batch(cuda_dev):
     tw = np.zeros((0, 2), np.float32)
     out = _run_mx(cuda_dev, x, W1, W2q, w2sf, ids, tw)
     assert out.shape == (0, 128)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "phi35", "qwen2", "wide2048"])
+def test_mx_layer_full_size_sampled(cuda_dev, name):
+    """The MX layer at full size, in the launch configuration the benchmark times:
+    the weight quantiser bit for bit over all of W2, and sampled tokens (every
+    expert's first and last slot, both sides of the heaviest and lightest experts'
+    m-tile boundaries, random ones) against the oracle's MX stages from x."""
+    from grouped_gemm_plan_b200 import workload as wl
+    from test_gpu_layer import _sample_tokens
+    w = wl.WORKLOADS[name]
+    dev = cuda_dev
+    x = wl.make_x(w)
+    W1 = torch.empty((w.E, w.H, 2 * w.F), dtype=torch.bfloat16, device=dev)
+    W2 = torch.empty((w.E, w.F, w.H), dtype=torch.bfloat16, device=dev)
+    wl.make_weights(w, W1, W2)
+    ids, tw = wl.make_routing(w)
+    W2q, w2sf = _mx_weights(dev, W2)
+    rq, rsf = oracle.mx_quantize_cols(W2.cpu())
+    assert np.array_equal(w2sf.cpu().numpy(), rsf) and np.array_equal(W2q.cpu().numpy(), rq)
+    out = _run_mx(dev, x, W1, W2q, w2sf, ids, tw)
+    counts, offsets, perm, inv, _ = oracle.plan(ids, tw, w.E)
+    tokens = _sample_tokens(ids, perm, offsets, 64, w.seed)
+    # the sampled (token, k) rows grouped by expert, through the oracle's stages
+    rows = sorted(((int(ids[t, k]), int(t), k) for t in tokens for k in range(w.topk)))
+    sub_counts = np.bincount([e for e, _, _ in rows], minlength=w.E)
+    sub_off = np.concatenate([[0], np.cumsum(sub_counts)]).astype(np.int32)
+    xs = x[torch.tensor([t for _, t, _ in rows])]
+    h = oracle.swiglu(oracle.grouped_gemm(xs, W1.cpu(), sub_off))
+    hq, hsf = oracle.mx_quantize_rows(h)
+    y = oracle.grouped_gemm_mx(hq, hsf, rq, rsf, sub_off)
+    pos = {t: j for j, t in enumerate(tokens)}
+    ref = np.zeros((len(tokens), w.H))
+    for (e, t, k), yr in sorted(zip(rows, y), key=lambda r: (r[0][1], r[0][2])):   # k ascending
+        ref[pos[t]] += float(tw[t, k]) * yr
+    check_close(out.cpu()[torch.from_numpy(tokens)], ref, f"{name} MX sampled rows")
