@@ -140,7 +140,7 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self._nvml = pynvml
-            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            h = self._nvml_handle(pynvml)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self._thread = threading.Thread(target=self._poll_nvml, args=(h,), daemon=True)
             self._thread.start()
@@ -158,6 +158,21 @@ class ClockSampler:
             self._thread.start()
         except OSError:
             self._proc = None
+
+    def _nvml_handle(self, nv):
+        """The NVML handle of the CUDA device this rank runs on: matched by UUID,
+        since NVML numbers every GPU of the machine while CUDA numbers only the
+        visible ones; by index when the UUID is not available."""
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.matched = "uuid " + uuid
+            return h
+        except Exception:
+            self.matched = f"index {self.index}"
+            return nv.nvmlDeviceGetHandleByIndex(self.index)
 
     def _poll_nvml(self, h):
         nv = self._nvml
@@ -201,7 +216,8 @@ class ClockSampler:
             return {"sm_mhz": statistics.median(mhz) if mhz else None,
                     "sm_mhz_min": min(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
                     "power_w_max": max(watts) if watts else None,
-                    "reasons": sorted(reasons), "samples": len(mhz), "source": "nvml 5 ms"}
+                    "reasons": sorted(reasons), "samples": len(mhz), "source": "nvml 5 ms",
+                    "nvml_device": getattr(self, "matched", None)}
         sm, smax = [], []
         for line in self._lines:
             parts = [p.strip() for p in line.split(",")]
