@@ -59,21 +59,32 @@ class ExpertShard:
 
 
 class CudaOps:
-    """The stage calls on this rank's GPU: the library's kernels through the C ABI."""
+    """The stage calls on this rank's GPU: the library's kernels through the C ABI.
+
+    Workspaces are kept per (call, sizes) and reused.  The calls are asynchronous on
+    the current stream; check() synchronises once and raises if any kernel recorded
+    a device error (ep_moe_ffn calls it at the end of the layer)."""
 
     def __init__(self, device):
         from . import binding as B
         self.B = B
         self.dev = torch.device(device)
+        self._cache = {}
         B.load()
 
     def _ws(self, op, M, H, F, E, topk):
-        return self.B.alloc_workspace(op, M, H, F, E, topk, self.dev)
+        key = (op, M, H, F, E, topk)
+        ws = self._cache.get(key)
+        if ws is None:
+            ws = self._cache[key] = self.B.alloc_workspace(op, M, H, F, E, topk, self.dev)
+        return ws
 
-    def _check(self, ws, what):
-        st = self.B.moe_get_device_status(ws)
-        if st != self.B.MOE_OK:
-            raise self.B.MoEError(st, f"device status after {what}")
+    def check(self):
+        """Synchronise; raise MoEError if a stage call recorded a device error."""
+        for key, ws in self._cache.items():
+            st = self.B.moe_get_device_status(ws)
+            if st != self.B.MOE_OK:
+                raise self.B.MoEError(st, f"device status of stage call {key[0]}")
 
     def plan(self, ids, E):
         """counts [E], offsets [E+1], perm [n*k], inv [n*k] of int32 ids [n, k]."""
@@ -85,7 +96,6 @@ class CudaOps:
         inv = torch.empty(max(n * k, 1), dtype=torch.int32, device=dev)
         ws = self._ws(B.OP_PLAN, n, 0, 0, E, k)
         B.moe_plan(ids, None, E, counts, offsets, perm[:n * k], inv[:n * k], None, ws)
-        self._check(ws, "the plan")
         return counts, offsets, perm[:n * k], inv[:n * k]
 
     def gather(self, rows, idx, topk=1):
@@ -96,7 +106,6 @@ class CudaOps:
             return out
         ws = self._ws(B.OP_DISPATCH, rows.shape[0], rows.shape[1], 0, 1, topk)
         B.moe_dispatch(rows, idx, topk, out, ws)
-        self._check(ws, "a gather")
         return out
 
     def expert_ffn(self, rows, offsets, W1, W2):
@@ -111,7 +120,6 @@ class CudaOps:
         ws = self._ws(B.OP_GROUPED_GEMM, n, 0, 0, E, 1)
         B.moe_grouped_gemm(rows, W1, offsets, B.EPI_SWIGLU, h, ws)
         B.moe_grouped_gemm(h, W2, offsets, B.EPI_STORE, y, ws)
-        self._check(ws, "the expert GEMMs")
         return y
 
     def combine(self, y, inv, topk_w):
@@ -121,7 +129,6 @@ class CudaOps:
         out = torch.empty((M, y.shape[1]), dtype=torch.bfloat16, device=self.dev)
         ws = self._ws(B.OP_COMBINE, M, y.shape[1], 0, 1, k)
         B.moe_combine(y, inv, topk_w, M, k, out, ws)
-        self._check(ws, "the combine")
         return out
 
 
@@ -188,7 +195,7 @@ def ep_moe_ffn(x, W1_local, W2_local, topk_ids, topk_w, shard: ExpertShard, ops,
     sent = ep_send(x, topk_ids, shard, ops)
     if G == 1:
         y = ep_experts(sent.xp, sent.send_counts.cpu().numpy(), W1_local, W2_local, ops)
-        return ep_finish(y, sent, topk_w, ops)
+        return _checked(ep_finish(y, sent, topk_w, ops), ops)
 
     recv_counts = torch.empty_like(sent.send_counts)
     dist.all_to_all_single(recv_counts, sent.send_counts, group=group)
@@ -201,4 +208,12 @@ def ep_moe_ffn(x, W1_local, W2_local, topk_ids, topk_w, shard: ExpertShard, ops,
     back = y.new_empty((sent.xp.shape[0], H))
     dist.all_to_all_single(back, y, output_split_sizes=send_rows, input_split_sizes=recv_rows,
                            group=group)
-    return ep_finish(back, sent, topk_w, ops)
+    return _checked(ep_finish(back, sent, topk_w, ops), ops)
+
+
+def _checked(out, ops):
+    """Run the stage calls' error check, where `ops` has one."""
+    check = getattr(ops, "check", None)
+    if check is not None:
+        check()
+    return out
