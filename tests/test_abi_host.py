@@ -189,6 +189,51 @@ def test_fp8_validation(lib):
     assert f(*fa(ws=need - 1)) == 4
 
 
+def test_mx_validation(lib):
+    qw = lib.moe_quantize_weights_mx
+    assert qw(FAKE, 0, 64, 64, FAKE, FAKE, None) == 2               # E
+    assert qw(FAKE, 2, 48, 64, FAKE, FAKE, None) == 2               # K % 32
+    assert qw(FAKE, 2, 64, 40, FAKE, FAKE, None) == 2               # N % 16
+    assert qw(FAKE, 2, 64, 64, FAKE, None, None) == 1               # null sf
+    assert qw(ctypes.c_void_p(0x10008), 2, 64, 64, FAKE, FAKE, None) == 7
+    qr = lib.moe_quantize_rows_mx
+    assert qr(FAKE, 4, 48, FAKE, FAKE, None) == 2                   # K % 32
+    assert qr(FAKE, -1, 64, FAKE, FAKE, None) == 1
+    assert qr(FAKE, 4, 64, None, FAKE, None) == 1
+    assert qr(None, 0, 64, None, None, None) == 0                   # R = 0: no-op
+    sw = lib.moe_grouped_gemm_swiglu_mx
+    swa = lambda **kw: [kw.get("A", FAKE), FAKE, FAKE, kw.get("E", 4), kw.get("R", 64),
+                        kw.get("K", 128), kw.get("N2", 256), FAKE, kw.get("sf", FAKE), FAKE_WS,
+                        256, None]
+    assert sw(*swa(N2=192)) == 2                                    # N2 % 128
+    assert sw(*swa(K=96)) == 2                                      # K % 64
+    assert sw(*swa(E=0)) == 2
+    assert sw(*swa(A=None)) == 1
+    assert sw(*swa(sf=ctypes.c_void_p(0x10001))) == 7               # 2-byte scale stores
+    g = lib.moe_grouped_gemm_mx
+    need = B.moe_workspace_size(B.OP_GEMM_MX, 64, 256, 128, 4, 1)
+    assert need >= 256 + (64 // 256 + 4) * 2 * 1 * 512 + 4 * 1 * 1 * 2 * 512
+    ga = lambda **kw: [kw.get("A", FAKE), FAKE, FAKE, FAKE, FAKE, kw.get("E", 4), kw.get("R", 64),
+                       kw.get("K", 128), kw.get("N", 256), None, None, FAKE, FAKE_WS,
+                       kw.get("ws", need), None]
+    assert g(*ga(K=48)) == 2                                        # K % 32
+    assert g(*ga(N=96)) == 2                                        # N % 64
+    assert g(*ga(R=-1)) == 1
+    assert g(*ga(A=None)) == 1
+    assert g(*ga(ws=need - 1)) == 4
+    assert g(*ga(A=ctypes.c_void_p(0x10008))) == 7
+    f = lib.moe_ffn_fused_mx
+    fneed = B.moe_workspace_size(B.OP_FFN_MX, 16, 128, 128, 4, 2)
+    fa = lambda **kw: [FAKE, FAKE, FAKE, kw.get("sf", FAKE), FAKE, FAKE, kw.get("M", 16),
+                       kw.get("H", 128), kw.get("F", 128), kw.get("E", 4), kw.get("topk", 2), FAKE,
+                       FAKE, FAKE, FAKE, FAKE_WS, kw.get("ws", fneed), None]
+    assert f(*fa(H=100)) == 2
+    assert f(*fa(F=96)) == 2
+    assert f(*fa(topk=5)) == 1
+    assert f(*fa(sf=None)) == 1
+    assert f(*fa(ws=fneed - 1)) == 4
+
+
 def test_stage_events_switch(lib):
     # off is always accepted; no CUDA call is made until a layer runs
     assert lib.moe_set_stage_events(None) == 0

@@ -358,3 +358,23 @@ def test_mx_layer_full_size_sampled(cuda_dev, name):
     ref = combine_rows(oracle.grouped_gemm_mx(hq, hsf, rq, rsf, sub_off))
     g = got.double().numpy()
     assert np.linalg.norm(g - ref) / np.linalg.norm(ref) < 1e-2
+
+
+def test_mx_layer_bad_expert_id(cuda_dev):
+    """An expert id out of range: the plan records MOE_ERR_BAD_EXPERT_ID and writes
+    zero counts; the GEMMs then have no rows and the call completes."""
+    w, x, W1, W2, ids, tw = layer_case(100, 128, 128, 4, 2, "uniform", seed=1)
+    ids = ids.copy()
+    ids[17, 0] = 4
+    dev = cuda_dev
+    W2q, w2sf = _mx_weights(dev, W2)
+    M, H = x.shape
+    out = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+    counts = torch.empty(4, dtype=torch.int32, device=dev)
+    offsets = torch.empty(5, dtype=torch.int32, device=dev)
+    perm = torch.empty(200, dtype=torch.int32, device=dev)
+    ws = B.alloc_workspace(B.OP_FFN_MX, M, H, 128, 4, 2, dev)
+    B.moe_ffn_fused_mx(x.to(dev), W1.to(dev), W2q, w2sf, torch.from_numpy(ids).to(dev),
+                       torch.from_numpy(tw).to(dev), out, counts, offsets, perm, ws)
+    assert B.moe_get_device_status(ws) == B.MOE_ERR_BAD_EXPERT_ID
+    assert counts.cpu().tolist() == [0] * 4
