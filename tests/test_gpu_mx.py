@@ -1,10 +1,11 @@
 """GPU parity of the block-scaled (MX) E4M3 down projection with the oracle: both
 quantisers bit for bit (codes and scale codes), the MX grouped GEMM within the
 fp32 summation bound, the SwiGLU epilogue's in-register quantisation against
-the oracle's quantiser applied to the exact h, and the MX layer against the
-oracle's MX layer (the bf16 layer's bar) and bit for bit against the chain of
-separate calls (which reaches the scale layout of the fused layer by another
-route)."""
+the oracle's quantiser applied to the exact h, and the MX layer element by element
+against the oracle's MX stages on the GPU's quantised h (the bf16 layer's bar),
+against the oracle's MX layer from x by relative Frobenius, and bit for bit against
+the chain of separate calls (which reaches the scale layout of the fused layer by
+another route)."""
 import numpy as np
 import pytest
 import torch
